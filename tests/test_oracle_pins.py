@@ -1,0 +1,300 @@
+"""Pins of the float64 oracle against facts fixed by the mathematics and by the method's
+statement, not against the oracle itself.
+
+The Light Forcing pages print no worked example of hierarchical sparse attention, so the
+pins are closed forms, brute force on tiny inputs, library routines for the special cases
+the method reduces to, and invariants the method's description implies:
+
+* pooling: ramp inputs whose block and frame means are known in closed form;
+* frame score linearity: a frame's pooled key is the length-weighted mean of its block
+  means, so its score is the length-weighted mean of block scores;
+* selection: exhaustive search over all k-subsets (maximal score sum, lexicographically
+  smallest among equals) agrees with the top-k rule;
+* attention: with every frame and block kept, HSA is full attention, checked against
+  torch's scaled_dot_product_attention in float64; zero queries give the uniform
+  average of the key set's values and lse = log(|key set|); probabilities are
+  non-negative and sum to one; unselected keys can be permuted or replaced freely;
+* fixed complexity: the number of selected blocks does not depend on the history length.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import lf_workloads as W
+from oracle import hsa64 as O
+
+
+# ------------------------------------------------------------------ pooling
+def _ramp_inputs(T=20, B=8, H=2, d=4, F=3, Fc=2, n_slots=5):
+    """q[t] = t (token index in the chunk), k in slot s at token t = 10*s + t/4.
+    All values are exact in bf16 (multiples of 1/4 below 64)."""
+    q = torch.zeros(Fc * T, H, d)
+    for t in range(Fc * T):
+        q[t] = float(t)
+    kc = torch.zeros(n_slots, T, H, d)
+    for s in range(n_slots):
+        for t in range(T):
+            kc[s, t] = 10.0 * s + t / 4.0
+    return q.to(torch.bfloat16), kc.to(torch.bfloat16)
+
+
+def test_block_bounds_closed_form():
+    b = O.block_bounds(1560, 64)
+    assert len(b) == 25 and b[-1] == (1536, 1560)          # 24 full blocks + 24 tokens
+    assert all(e - s == 64 for s, e in b[:-1])
+    assert sum(e - s for s, e in b) == 1560
+    assert O.block_bounds(1560, 128)[-1] == (1536, 1560) and O.n_blocks(1560, 128) == 13
+    assert O.block_bounds(256, 64) == [(0, 64), (64, 128), (128, 192), (192, 256)]
+
+
+def test_pooling_ramp_closed_form():
+    T, B = 20, 8
+    q, kc = _ramp_inputs(T, B)
+    qb = O.compress_queries(q, T, B)
+    # blocks of frame f: [0,8), [8,16), [16,20) -> mean token = f*T + (s + e - 1)/2
+    for f in range(2):
+        for b, (s, e) in enumerate([(0, 8), (8, 16), (16, 20)]):
+            assert np.allclose(qb[:, f * 3 + b, :], f * T + (s + e - 1) / 2.0, atol=0, rtol=0)
+    slots = [3, 0, 4]
+    kb, kf = O.compress_keys(kc, slots, T, B)
+    for f, s in enumerate(slots):
+        for b, (a, e) in enumerate([(0, 8), (8, 16), (16, 20)]):
+            assert np.allclose(kb[:, f, b, :], 10.0 * s + (a + e - 1) / 8.0, rtol=0, atol=1e-12)
+        assert np.allclose(kf[:, f, :], 10.0 * s + (T - 1) / 8.0, rtol=0, atol=1e-12)
+
+
+def test_frame_pool_is_length_weighted_block_mean():
+    ci = W.random_small(3, H=2, d=16, T=100, block=32, n_cur_frames=1, n_hist=3,
+                        n_sink=0, k_f=2, k_b=2)
+    kb, kf = O.compress_keys(ci.k_cache, ci.hist_slots, ci.shape.T, ci.shape.block)
+    lens = np.array([e - s for s, e in O.block_bounds(100, 32)], dtype=np.float64)
+    lin = np.einsum("hfbd,b->hfd", kb, lens) / 100.0
+    assert np.allclose(lin, kf, rtol=0, atol=1e-12)
+    # so the frame score equals the length-weighted mean of block scores
+    qb = O.compress_queries(ci.q, 100, 32)
+    sf = O.frame_scores(qb, kf)
+    sb_all = np.einsum("hqd,hfbd->hqfb", qb, kb)
+    assert np.allclose(sf, np.einsum("hqfb,b->hqf", sb_all, lens) / 100.0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ selection
+def _brute_topk(scores, k):
+    """Exhaustive: the k-subset with the largest score sum; among equal sums the
+    lexicographically smallest index tuple (ties to lower indices)."""
+    best, best_key = None, None
+    for sub in itertools.combinations(range(len(scores)), k):
+        key = (-sum(scores[i] for i in sub), sub)
+        if best_key is None or key < best_key:
+            best, best_key = sub, key
+    return list(best)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_topk_matches_brute_force(seed):
+    g = np.random.default_rng(seed)
+    n = int(g.integers(1, 9))
+    k = int(g.integers(1, n + 1))
+    if seed % 2:
+        scores = list(g.integers(-2, 3, size=n).astype(float))   # many exact ties
+    else:
+        scores = list(g.standard_normal(n))
+    assert O.topk_lower_index(scores, k) == _brute_topk(scores, k)
+
+
+def test_topk_ties_go_to_lower_index():
+    assert O.topk_lower_index([1.0, 2.0, 2.0, 2.0, 0.5], 2) == [1, 2]
+    assert O.topk_lower_index([5.0, 5.0, 5.0], 1) == [0]
+    assert O.topk_lower_index([-1.0, -1.0, 3.0], 2) == [0, 2]
+    assert O.topk_lower_index([0.0, 1.0], 5) == [0, 1]        # k >= n keeps everything
+
+
+def test_boundary_gap_closed_form():
+    assert O.boundary_gap([4.0, 1.0, 3.0, 2.0], 2) == pytest.approx((3.0 - 2.0) / 3.0)
+    assert O.boundary_gap([1.0, 2.0], 2) == math.inf
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_two_stage_selection_brute_force(seed):
+    """Frames, then blocks inside each chosen frame, against exhaustive search with the
+    scores recomputed through a different route (reshape-mean pooling + einsum)."""
+    g = np.random.default_rng(100 + seed)
+    T, B = int(g.choice([40, 48, 50])), 16
+    F, kf, kb = int(g.integers(2, 6)), int(g.integers(1, 3)), int(g.integers(1, 3))
+    ci = W.random_small(seed, H=2, d=8, T=T, block=B, n_cur_frames=1, n_hist=F,
+                        n_sink=0, k_f=kf, k_b=kb)
+    qb = O.compress_queries(ci.q, T, B)
+    kbk, kfr = O.compress_keys(ci.k_cache, ci.hist_slots, T, B)
+    fidx, _ = O.select_frames(qb, kfr, kf)
+    bidx, _ = O.select_blocks(qb, kbk, fidx, kb)
+
+    q64 = ci.q.double().numpy()
+    k64 = ci.k_cache.double().numpy()
+    nb = -(-T // B)
+    pad = nb * B - T
+    kfr2 = np.stack([k64[s].mean(axis=0) for s in ci.hist_slots], axis=1)      # [H,F,d]
+    for h in range(2):
+        for qi in range(nb):
+            s, e = qi * B, min(qi * B + B, T)
+            qv = q64[s:e, h, :].mean(axis=0)
+            fs = [float(qv @ kfr2[h, f]) for f in range(F)]
+            frames = _brute_topk(fs, min(kf, F))
+            assert list(fidx[h, qi]) == frames
+            want = []
+            for f in frames:
+                fr = k64[ci.hist_slots[f], :, h, :]
+                means = [fr[b * B:min(b * B + B, T)].mean(axis=0) for b in range(nb)]
+                bs = [float(qv @ m) for m in means]
+                want += [f * nb + b for b in _brute_topk(bs, min(kb, nb))]
+            assert list(bidx[h, qi]) == sorted(want)
+
+
+def test_fixed_complexity_independent_of_history_length():
+    counts = set()
+    for F in (3, 6, 12):
+        ci = W.random_small(F, H=2, d=8, T=64, block=16, n_cur_frames=1, n_hist=F,
+                            n_sink=0, k_f=2, k_b=3)
+        r = O.forward_chunk(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                            ci.hist_slots, ci.sink_slots)
+        counts.add(r["block_idx"].shape[-1])
+        assert r["frame_idx"].shape[-1] == 2
+    assert counts == {2 * 3}
+
+
+def test_planted_frame_recovered():
+    """Soft check: queries pulled towards one history frame usually select it."""
+    ci = W.random_small(11, H=4, d=64, T=256, block=64, n_cur_frames=2, n_hist=8,
+                        n_sink=0, k_f=2, k_b=2)
+    qb = O.compress_queries(ci.q, 256, 64)
+    _, kfr = O.compress_keys(ci.k_cache, ci.hist_slots, 256, 64)
+    fidx, _ = O.select_frames(qb, kfr, 2)
+    hits = [ci.planted[h, qi // 4] in fidx[h, qi] for h in range(4) for qi in range(8)]
+    assert np.mean(hits) >= 0.8
+
+
+# ------------------------------------------------------------------ attention
+def _dense_reference_sdpa(ci):
+    """torch SDPA (float64, CPU) over current + sinks + all history frames."""
+    sh = ci.shape
+    keys = [ci.k_cur.double()] + [ci.k_cache[s].double() for s in ci.sink_slots] + \
+           [ci.k_cache[s].double() for s in ci.hist_slots]
+    vals = [ci.v_cur.double()] + [ci.v_cache[s].double() for s in ci.sink_slots] + \
+           [ci.v_cache[s].double() for s in ci.hist_slots]
+    K = torch.cat(keys, 0).permute(1, 0, 2)[None]
+    V = torch.cat(vals, 0).permute(1, 0, 2)[None]
+    Q = ci.q.double().permute(1, 0, 2)[None]
+    out = torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=sh.scale)
+    logits = torch.einsum("hqd,hkd->hqk", Q[0], K[0]) * sh.scale
+    return out[0].permute(1, 0, 2).numpy(), torch.logsumexp(logits, -1).numpy()
+
+
+@pytest.mark.parametrize("T,B,F,S", [(100, 32, 3, 0), (96, 32, 2, 1), (64, 64, 1, 2)])
+def test_dense_equivalence_with_sdpa(T, B, F, S):
+    ci = W.random_small(T + F, H=2, d=16, T=T, block=B, n_cur_frames=2, n_hist=F,
+                        n_sink=S, k_f=F, k_b=-(-T // B))
+    r = O.forward_chunk(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                        ci.hist_slots, ci.sink_slots)
+    o_ref, lse_ref = _dense_reference_sdpa(ci)
+    assert np.allclose(r["O"], o_ref, rtol=0, atol=1e-12)
+    assert np.allclose(r["lse"], lse_ref, rtol=0, atol=1e-12)
+
+
+def test_no_history_is_attention_over_current_and_sinks():
+    ci = W.random_small(5, H=2, d=16, T=48, block=16, n_cur_frames=2, n_hist=0,
+                        n_sink=2, k_f=1, k_b=1)
+    r = O.forward_chunk(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                        ci.hist_slots, ci.sink_slots)
+    o_ref, _ = _dense_reference_sdpa(ci)
+    assert np.allclose(r["O"], o_ref, rtol=0, atol=1e-12)
+
+
+def test_zero_queries_average_values_and_lse_counts_keys():
+    """q = 0 gives equal logits: O is the plain mean of the key set's values and
+    lse = log(number of keys) = log(F_c*T + S*T + sum of selected block lengths)."""
+    ci = W.random_small(7, H=2, d=16, T=50, block=16, n_cur_frames=1, n_hist=4,
+                        n_sink=1, k_f=2, k_b=2)
+    sh = ci.shape
+    r = O.forward_chunk(sh, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                        ci.hist_slots, ci.sink_slots)
+    bidx = r["block_idx"]
+    zq = torch.zeros_like(ci.q)
+    O0, lse0 = O.attention(sh, zq, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                           ci.hist_slots, ci.sink_slots, bidx)
+    nb = 4                       # blocks of 16 over 50 tokens: 16, 16, 16, 2
+    lens = [16, 16, 16, 2]
+    v64 = ci.v_cache.double().numpy()
+    vc64 = ci.v_cur.double().numpy()
+    for h in range(2):
+        for qi in range(nb):
+            sel = [int(g) for g in bidx[h, qi]]
+            n_keys = 50 + 50 + sum(lens[g % nb] for g in sel)
+            total = vc64[:, h].sum(0) + v64[ci.sink_slots[0], :, h].sum(0)
+            for g in sel:
+                f, b = divmod(g, nb)
+                total = total + v64[ci.hist_slots[f], b * 16:b * 16 + lens[b], h].sum(0)
+            rows = slice(qi * 16, qi * 16 + lens[qi])
+            assert np.allclose(O0[rows, h], total / n_keys, rtol=0, atol=1e-12)
+            assert np.allclose(lse0[h, rows], math.log(n_keys), rtol=0, atol=1e-12)
+
+
+def test_two_key_closed_form():
+    """One query, two keys with logits 0 and x: O = (v0 + e^x v1) / (1 + e^x)."""
+    q = np.array([[1.0, 0.0]])
+    k = np.array([[0.0, 1.0], [2.0, 0.0]])
+    v = np.array([[1.0, 0.0], [0.0, 1.0]])
+    o, lse, P = O.attention_qblock(q, k, v, 0.5)
+    x = 1.0
+    assert np.allclose(o, [[1 / (1 + math.e ** x), math.e ** x / (1 + math.e ** x)]], atol=1e-15)
+    assert np.allclose(lse, [math.log(1 + math.e ** x)], atol=1e-15)
+
+
+def test_probabilities_are_a_distribution():
+    g = np.random.default_rng(0)
+    q, k, v = g.standard_normal((7, 32)), g.standard_normal((300, 32)) * 3, g.standard_normal((300, 32))
+    _, _, P = O.attention_qblock(q, k, v, 1 / math.sqrt(32))
+    assert (P >= 0).all()
+    assert np.abs(P.sum(axis=1) - 1.0).max() < 1e-12
+
+
+def test_unselected_blocks_do_not_matter():
+    """Replacing every unselected history block (contents permuted across tokens and
+    scaled) leaves O unchanged for a fixed selection; touching one selected block
+    changes it."""
+    ci = W.random_small(9, H=2, d=16, T=64, block=16, n_cur_frames=1, n_hist=4,
+                        n_sink=0, k_f=2, k_b=2)
+    sh = ci.shape
+    r = O.forward_chunk(sh, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                        ci.hist_slots, ci.sink_slots)
+    bidx = r["block_idx"]
+    nb = 4
+    for h in range(2):
+        for qi in range(nb):
+            sel = set(int(g) for g in bidx[h, qi])
+            kc, vc = ci.k_cache.clone(), ci.v_cache.clone()
+            g = torch.Generator().manual_seed(h * 10 + qi)
+            for f, slot in enumerate(ci.hist_slots):
+                for b in range(nb):
+                    if f * nb + b not in sel:
+                        perm = torch.randperm(16, generator=g) + b * 16
+                        kc[slot, b * 16:(b + 1) * 16, h] = (kc[slot, perm, h].float() * 2).bfloat16()
+                        vc[slot, b * 16:(b + 1) * 16, h] = (vc[slot, perm, h].float() * -3).bfloat16()
+            O2, _ = O.attention(sh, ci.q, ci.k_cur, ci.v_cur, kc, vc, ci.hist_slots,
+                                ci.sink_slots, bidx, heads=[h], qblocks=[qi])
+            rows = slice(qi * 16, (qi + 1) * 16)
+            assert np.array_equal(O2[rows, h], r["O"][rows, h])
+            f, b = divmod(min(sel), nb)
+            vc[ci.hist_slots[f], b * 16, h] += 1.0
+            O3, _ = O.attention(sh, ci.q, ci.k_cur, ci.v_cur, kc, vc, ci.hist_slots,
+                                ci.sink_slots, bidx, heads=[h], qblocks=[qi])
+            assert not np.allclose(O3[rows, h], r["O"][rows, h], rtol=0, atol=1e-9)
+
+
+def test_executed_flops_counts_valid_pairs():
+    """4*d per (query, key) pair; at full selection this is 4*d*Nq*(all keys)."""
+    ci = W.random_small(2, H=2, d=16, T=50, block=16, n_cur_frames=2, n_hist=3,
+                        n_sink=1, k_f=3, k_b=4)
+    r = O.forward_chunk(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                        ci.hist_slots, ci.sink_slots)
+    assert O.executed_flops(ci.shape, r["block_idx"]) == 4 * 16 * 2 * 100 * (100 + 50 + 150)
