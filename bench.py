@@ -1,0 +1,368 @@
+"""Benchmark of the hierarchical sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lf|reference] [--config 480p]
+
+One step = one pass of the whole path over one synthetic chunk: (a) token compression,
+(b) frame top-k, (c) block top-k, (d) block-sparse attention, each through its C-ABI
+entry point (lf_compress, lf_select_frames, lf_select_blocks, lf_block_sparse_attn) on
+inputs already resident in HBM.  The L2 cache is flushed (a 256 MB write) before every
+timed step, outside the step's event pair.  Reported: effective TFLOP/s = executed
+attention FLOPs (4*d per valid query-key pair) / step time; ms per chunk; roofline of the
+dominant kernel (attention, bf16 tensor cores) and of the selection (HBM); the e2e
+figure through lf_forward_chunk with host buffers (pinned host -> device copy of the
+chunk's Q/K/V, device -> host copy of the output inside the timed region; the KV cache is
+state that stays resident); and the float64 oracle timed on the host cores on a bounded
+sample.
+
+Multi-GPU (torchrun): every rank runs its own chunk (independent video streams), no
+collective on the data path; value = all ranks' FLOPs / max-over-ranks time (weak
+scaling).  --impl reference times the float64 CPU oracle on the same config (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def block_lens(T, B):
+    nb = -(-T // B)
+    return np.array([min(B, T - b * B) for b in range(nb)], dtype=np.int64)
+
+
+def executed_flops(shape, block_idx_np) -> int:
+    """4*d per (head, query, valid key): current chunk + sinks dense, plus the tokens of the
+    selected blocks of each query's block."""
+    lens = block_lens(shape.T, shape.block)
+    nb = len(lens)
+    qlen = np.tile(lens, shape.n_cur_frames)                  # tokens per query block
+    dense = shape.n_cur_frames * shape.T + shape.n_sink * shape.T
+    sel = np.zeros((shape.H, len(qlen)), dtype=np.int64)
+    if shape.n_hist > 0 and block_idx_np is not None:
+        sel = lens[block_idx_np % nb].sum(axis=-1)
+    return int(4 * shape.d * (qlen[None, :] * (dense + sel)).sum())
+
+
+def selection_bytes(shape) -> int:
+    return 2 * shape.H * shape.d * shape.T * (shape.n_cur_frames + shape.n_hist)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.6)
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [l for (t, l) in self.lines if t0 - 0.15 <= t <= t1 + 0.15] or \
+               [l for (_, l) in self.lines]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in rows:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def make_workload(name, seed):
+    import lf_workloads as W
+    if name == "480p":
+        return W.p480(seed), "Self-Forcing-shaped 480p chunk: H=12 d=128 T=1560 (30x52), " \
+                             "chunk 3 frames (4680 queries), 18 history frames, B=64, k_f=6, k_b=12"
+    if name == "large":
+        return W.large(seed), "large-model stress: H=40 d=128 T=1560, chunk 3, " \
+                              "42 history frames, B=128, k_f=8, k_b=5"
+    raise SystemExit(f"unknown config {name}")
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_sample(ci, budget_s=0.0, first_head=0):
+    """Runs the float64 oracle (a)-(d) head by head (each head is an independent problem)
+    until `budget_s` seconds are spent (at least one head): a bounded sample of the chunk.
+    Returns (executed FLOPs of the sample, seconds, cores, heads run)."""
+    from dataclasses import replace
+    from oracle import hsa64 as O
+    import torch
+    sh = ci.shape
+    s1 = replace(sh, H=1)
+    flops, dt, heads = 0, 0.0, 0
+    for i in range(sh.H):
+        h = (first_head + i) % sh.H
+        sl = lambda t: t[..., h:h + 1, :].contiguous()
+        t0 = time.perf_counter()
+        r = O.forward_chunk(s1, sl(ci.q), sl(ci.k_cur), sl(ci.v_cur), sl(ci.k_cache),
+                            sl(ci.v_cache), ci.hist_slots, ci.sink_slots)
+        dt += time.perf_counter() - t0
+        flops += executed_flops(s1, r.get("block_idx"))
+        heads += 1
+        if dt >= budget_s:
+            break
+    return flops, dt, torch.get_num_threads(), heads
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    ci, desc = make_workload(args.config, 0)
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(ci)
+    tot_f, tot_t, cores = 0, 0.0, 1
+    for k in range(args.steps):
+        f, t, cores, _ = oracle_sample(ci, first_head=k)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    sample = f"one head of the {args.config} chunk per step ((a)-(d), float64 numpy)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc, "oracle_sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "ms/chunk & effective TFLOP/s, hierarchical sparse attn, 480p chunk shape"
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_lf(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import block_sparse_attention_46_b200 as lf
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lf.load()
+    ci, desc = make_workload(args.config, rank)
+    sh = ci.shape
+    nbpf, nqb, kf, kb = lf.derived(sh)
+    t = {k: getattr(ci, k).to(dev) for k in ("q", "k_cur", "v_cur", "k_cache", "v_cache")}
+    q_blk = torch.empty(sh.H, nqb, sh.d, device=dev)
+    k_blk = torch.empty(sh.H, max(sh.n_hist, 1), nbpf, sh.d, device=dev)
+    k_frm = torch.empty(sh.H, max(sh.n_hist, 1), sh.d, device=dev)
+    fidx = torch.empty(sh.H, nqb, max(kf, 1), dtype=torch.int32, device=dev)
+    bidx = torch.empty(sh.H, nqb, max(kf * kb, 1), dtype=torch.int32, device=dev)
+    out = torch.empty_like(t["q"])
+    lse = torch.empty(sh.H, t["q"].shape[0], device=dev)
+    ws = torch.empty(max(lf.lf_attn_workspace_size(sh), 256), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def step(record=False):
+        if record:
+            ev[0].record(stream)
+        lf.lf_compress(sh, t["q"], t["k_cache"], ci.hist_slots, q_blk, k_blk, k_frm)
+        lf.lf_select_frames(sh, q_blk, k_frm, fidx)
+        lf.lf_select_blocks(sh, q_blk, k_blk, fidx, bidx)
+        if record:
+            ev[1].record(stream)
+        lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
+                                ci.hist_slots, ci.sink_slots, bidx, out, lse, ws)
+        if record:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    flops = executed_flops(sh, bidx.cpu().numpy())
+    launches_per_step = 6 if sh.n_hist > 0 else 2
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    sel_ms, att_ms = [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        step(record=True)
+        ev[2].synchronize()
+        sel_ms.append(ev[0].elapsed_time(ev[1]))
+        att_ms.append(ev[1].elapsed_time(ev[2]))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall1 = time.time()
+    clk = clocks.stop(t_wall0, t_wall1)
+    assert lf.lf_device_status() == 0, "device status reported an error"
+
+    step_ms = [a + b for a, b in zip(sel_ms, att_ms)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_step = total_ms / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # e2e through lf_forward_chunk with host buffers
+    hq = {k: t[k].cpu().pin_memory() for k in ("q", "k_cur", "v_cur")}
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    fws = torch.empty(lf.lf_forward_workspace_size(sh), dtype=torch.uint8, device=dev)
+    n_e2e = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step():
+        for k in ("q", "k_cur", "v_cur"):
+            t[k].copy_(hq[k], non_blocking=True)
+        lf.lf_forward_chunk(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
+                            ci.hist_slots, ci.sink_slots, out, None, None, fws)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = sum(hq[k].numel() * hq[k].element_size() for k in hq)
+    d2h = hout.numel() * hout.element_size()
+
+    pk, src = peaks()
+    att_mean = statistics.mean(att_ms)
+    sel_mean = statistics.mean(sel_ms)
+    att_tflops = flops / (att_mean * 1e-3) / 1e12
+    sel_gbs = selection_bytes(sh) / (sel_mean * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; per-frame key centroids, planted related frames)",
+        "config": {"workload": desc, "l2": "flushed (256 MB write) before every timed step",
+                   "executed_gflop_per_chunk": flops / 1e9,
+                   "selection_mb_per_chunk": selection_bytes(sh) / 1e6,
+                   "ms_selection_abc": sel_mean, "ms_attention_d": att_mean,
+                   "selection_share": sel_mean / (sel_mean + att_mean)},
+        "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": att_tflops / pk["bf16_tflops"],
+                     "traffic": None, "kernel": "attn_kernel (+ plan_kernel) = stage (d)",
+                     "peak_source": f"{src} bf16_tflops (burst)"},
+        "roofline_selection": {"bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": sel_gbs / pk["hbm_gbs"],
+                               "kernels": "pool_blocks + pool_frames + select_frames + select_blocks",
+                               "peak_source": f"{src} hbm_gbs"},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "lf_forward_chunk"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, dt, cores, heads = oracle_sample(ci, budget_s=10.0)
+        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "seconds": dt,
+                                "sample": f"heads 0..{heads - 1} of {sh.H} of the chunk: "
+                                          f"(a)-(d) float64 numpy, head by head"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="lf", choices=["lf", "reference"])
+    ap.add_argument("--config", default="480p")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        args.steps = min(args.steps, 30)     # ~1 s of oracle work per step
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_lf(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

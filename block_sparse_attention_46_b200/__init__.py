@@ -1,0 +1,186 @@
+"""Python binding of liblf, the sm_100a hierarchical sparse attention library.
+
+Argument marshalling only: every function below forwards to the C entry point of the
+same name in ``liblf.so`` (declared in include/lf.h) with raw device pointers, host
+slot lists and the current CUDA stream.  PyTorch provides device memory and streams; no
+step of the attention path runs in Python or on the CPU.  If the library is missing or
+does not load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "LfError", "LfShape", "load", "make_shape", "lf_compress", "lf_select_frames",
+    "lf_select_blocks", "lf_block_sparse_attn", "lf_forward_chunk",
+    "lf_attn_workspace_size", "lf_forward_workspace_size", "lf_device_status",
+    "lf_status_string", "lf_abi_version", "derived", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblf.so")
+
+LF_OK = 0
+
+
+class LfError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: liblf status {code} ({lf_status_string(code)})")
+
+
+class LfShape(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("tokens_per_frame", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("n_cur_frames", ctypes.c_int32), ("n_hist", ctypes.c_int32),
+                ("n_sink", ctypes.c_int32), ("n_slots", ctypes.c_int32),
+                ("k_f", ctypes.c_int32), ("k_b", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_SHP = ctypes.POINTER(LfShape)
+
+_SIGS = {
+    "lf_compress": (ctypes.c_int, [_SHP, _P, _P, _I32P, _P, _P, _P, _P]),
+    "lf_select_frames": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P]),
+    "lf_select_blocks": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _P]),
+    "lf_attn_workspace_size": (_SZ, [_SHP]),
+    "lf_block_sparse_attn": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P, _P,
+                                            _P, _P, _SZ, _P]),
+    "lf_forward_workspace_size": (_SZ, [_SHP]),
+    "lf_forward_chunk": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P, _SZ, _P,
+                                        _P, _P, _P]),
+    "lf_device_status": (ctypes.c_int, [ctypes.c_int]),
+    "lf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "lf_abi_version": (ctypes.c_int, []),
+}
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads liblf.so (once) and declares its signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise FileNotFoundError(
+                f"{path} is missing: build it with python -m block_sparse_attention_46_b200.build")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = lib
+    return _lib
+
+
+def make_shape(s) -> LfShape:
+    """lf_shape from any object with the plain size fields (H, d, T, block, ...)."""
+    return LfShape(s.H, s.d, s.T, s.block, s.n_cur_frames, s.n_hist, s.n_sink, s.n_slots,
+                   s.k_f, s.k_b, s.scale)
+
+
+def derived(s):
+    """(n_bpf, n_qb, kf, kb) as the library derives them (for sizing output tensors)."""
+    nbpf = -(-s.T // s.block)
+    kf = min(s.k_f, s.n_hist) if s.n_hist > 0 else 0
+    kb = min(s.k_b, nbpf) if s.n_hist > 0 else 0
+    return nbpf, s.n_cur_frames * nbpf, kf, kb
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _slots(v: Sequence[int]):
+    arr = (ctypes.c_int32 * max(len(v), 1))(*[int(x) for x in v])
+    return ctypes.cast(arr, _I32P), arr          # keep `arr` alive during the call
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != LF_OK:
+        raise LfError(rc, where)
+
+
+def lf_status_string(code: int) -> str:
+    return load().lf_status_string(code).decode()
+
+
+def lf_abi_version() -> int:
+    return load().lf_abi_version()
+
+
+def lf_device_status(reset: bool = True) -> int:
+    return load().lf_device_status(1 if reset else 0)
+
+
+def lf_compress(shape, q, k_cache, hist_slots, q_blk, k_blk, k_frm, stream=None):
+    sh = make_shape(shape)
+    hs, _keep = _slots(hist_slots)
+    _check(load().lf_compress(ctypes.byref(sh), _ptr(q), _ptr(k_cache), hs, _ptr(q_blk),
+                              _ptr(k_blk), _ptr(k_frm), _stream(stream)), "lf_compress")
+
+
+def lf_select_frames(shape, q_blk, k_frm, frame_idx, frame_score=None, stream=None):
+    sh = make_shape(shape)
+    _check(load().lf_select_frames(ctypes.byref(sh), _ptr(q_blk), _ptr(k_frm), _ptr(frame_idx),
+                                   _ptr(frame_score), _stream(stream)), "lf_select_frames")
+
+
+def lf_select_blocks(shape, q_blk, k_blk, frame_idx, block_idx, block_score=None, stream=None):
+    sh = make_shape(shape)
+    _check(load().lf_select_blocks(ctypes.byref(sh), _ptr(q_blk), _ptr(k_blk), _ptr(frame_idx),
+                                   _ptr(block_idx), _ptr(block_score), _stream(stream)),
+           "lf_select_blocks")
+
+
+def lf_attn_workspace_size(shape) -> int:
+    sh = make_shape(shape)
+    return int(load().lf_attn_workspace_size(ctypes.byref(sh)))
+
+
+def lf_forward_workspace_size(shape) -> int:
+    sh = make_shape(shape)
+    return int(load().lf_forward_workspace_size(ctypes.byref(sh)))
+
+
+def lf_block_sparse_attn(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
+                         block_idx, out, lse=None, workspace=None, stream=None):
+    sh = make_shape(shape)
+    hs, _k1 = _slots(hist_slots)
+    ss, _k2 = _slots(sink_slots)
+    if workspace is None:
+        workspace = torch.empty(max(lf_attn_workspace_size(shape), 256), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().lf_block_sparse_attn(
+        ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_cache), _ptr(v_cache), hs, ss,
+        _ptr(block_idx), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "lf_block_sparse_attn")
+
+
+def lf_forward_chunk(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
+                     out, lse=None, block_idx_out=None, workspace=None, stream=None):
+    sh = make_shape(shape)
+    hs, _k1 = _slots(hist_slots)
+    ss, _k2 = _slots(sink_slots)
+    if workspace is None:
+        workspace = torch.empty(max(lf_forward_workspace_size(shape), 256), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().lf_forward_chunk(
+        ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_cache), _ptr(v_cache), hs, ss,
+        _ptr(workspace), workspace.numel(), _ptr(out), _ptr(lse), _ptr(block_idx_out),
+        _stream(stream)), "lf_forward_chunk")

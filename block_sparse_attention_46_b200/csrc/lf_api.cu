@@ -1,0 +1,358 @@
+// lf_api.cu — the C ABI of liblf (declared in include/lf.h): argument validation, launch
+// configuration and tensor-map set-up for the four hierarchical-sparse-attention stages.
+// The library is one translation unit: the kernels are included below.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <mutex>
+#include <string.h>
+
+#include "lf_common.cuh"
+#include "lf_select.cuh"
+#include "lf_attn.cuh"
+
+using lf::Dims;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Validates the plain sizes and derives the rest.  Returns LF_OK or an error code.
+int make_dims(const lf_shape* s, Dims* D) {
+  if (s == nullptr || D == nullptr) return LF_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return LF_ERR_UNSUPPORTED;
+  if (s->block != 64 && s->block != 128) return LF_ERR_UNSUPPORTED;
+  if (s->H < 1 || s->tokens_per_frame < 1 || s->n_cur_frames < 1 || s->n_hist < 0 ||
+      s->n_sink < 0 || s->n_slots < 0)
+    return LF_ERR_INVALID_ARG;
+  if (s->tokens_per_frame > LF_MAX_T) return LF_ERR_UNSUPPORTED;
+  if (s->n_hist + s->n_sink > LF_MAX_FRAMES) return LF_ERR_UNSUPPORTED;
+  if ((s->n_hist > 0 || s->n_sink > 0) && s->n_slots < 1) return LF_ERR_INVALID_ARG;
+  if (s->n_hist > 0 && (s->k_f < 1 || s->k_b < 1)) return LF_ERR_INVALID_ARG;
+  if (!(s->scale > 0.f) || s->scale > 1e30f) return LF_ERR_INVALID_ARG;
+  const long long ncur = (long long)s->n_cur_frames * s->tokens_per_frame;
+  if (ncur > (1LL << 30) / ((long long)s->H * s->d)) return LF_ERR_UNSUPPORTED;
+  if ((long long)s->n_slots * s->tokens_per_frame * s->H * s->d > (1LL << 40))
+    return LF_ERR_UNSUPPORTED;
+  Dims d{};
+  d.H = s->H; d.d = s->d; d.T = s->tokens_per_frame; d.B = s->block;
+  d.Fc = s->n_cur_frames; d.F = s->n_hist; d.S = s->n_sink; d.n_slots = s->n_slots;
+  d.nbpf = lf::cdiv(d.T, d.B);
+  d.nqb = d.Fc * d.nbpf;
+  d.ncur = d.Fc * d.T;
+  d.kf = d.F > 0 ? (s->k_f < d.F ? s->k_f : d.F) : 0;
+  d.kb = d.F > 0 ? (s->k_b < d.nbpf ? s->k_b : d.nbpf) : 0;
+  d.nsel = d.kf * d.kb;
+  d.scale = s->scale;
+  if (d.nsel > LF_MAX_SELECTED) return LF_ERR_UNSUPPORTED;
+  if (lf::plan_stride(d) > lf::kMaxPlan) return LF_ERR_UNSUPPORTED;
+  *D = d;
+  return LF_OK;
+}
+
+int check_slots(const int32_t* slots, int n, int n_slots) {
+  if (n == 0) return LF_OK;
+  if (slots == nullptr) return LF_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (slots[i] < 0 || slots[i] >= n_slots) return LF_ERR_INVALID_ARG;
+  return LF_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? LF_OK : LF_ERR_CUDA; }
+
+// --------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// bf16 rows of H*d channels: 2-D [rows, H*d] or 3-D [slots, T, H*d]; box = 64 channels x
+// 64 rows (x 1 slot); 128-byte swizzle; out-of-bounds elements read as zero.
+int encode_rows(CUtensorMap* m, const void* base, int HD, long long rows, int slots) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return LF_ERR_CUDA;
+  const cuuint32_t rank = slots > 0 ? 3 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)rows, (cuuint64_t)(slots > 0 ? slots : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)HD * 2 * (cuuint64_t)rows};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LF_OK : LF_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- launches
+int launch_compress(const Dims& D, const void* q, const void* k_cache, const int32_t* hist_slots,
+                    float* q_blk, float* k_blk, float* k_frm, cudaStream_t st) {
+  lf::PoolArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  a.q_blk = q_blk;
+  a.k_blk = k_blk;
+  for (int f = 0; f < D.F; ++f) a.hist_slots[f] = hist_slots[f];
+  const int units = D.nqb + D.F * D.nbpf;
+  const int vecs = D.H * D.d / 8;
+  dim3 grid(units, lf::cdiv(vecs, lf::kPoolThreads));
+  lf::pool_blocks_kernel<<<grid, lf::kPoolThreads, 0, st>>>(a, D);
+  if (D.F > 0) lf::pool_frames_kernel<<<dim3(D.F, D.H), D.d, 0, st>>>(k_blk, k_frm, D);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_select_frames(const Dims& D, const float* q_blk, const float* k_frm,
+                         int32_t* frame_idx, float* frame_score, cudaStream_t st) {
+  const size_t smem = ((size_t)D.F * (D.d + 4) + (size_t)lf::kSelWarps * D.d) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(lf::select_frames_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return LF_ERR_CUDA;
+  dim3 grid(lf::cdiv(D.nqb, lf::kSelWarps), D.H);
+  lf::select_frames_kernel<<<grid, lf::kSelWarps * 32, smem, st>>>(q_blk, k_frm, frame_idx,
+                                                                   frame_score, D);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_select_blocks(const Dims& D, const float* q_blk, const float* k_blk,
+                         const int32_t* frame_idx, int32_t* block_idx, float* block_score,
+                         cudaStream_t st) {
+  const size_t smem = ((size_t)D.nbpf * (D.d + 4) + (size_t)lf::kSelWarps * D.d) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(lf::select_blocks_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return LF_ERR_CUDA;
+  lf::select_blocks_kernel<<<dim3(D.F, D.H), lf::kSelWarps * 32, smem, st>>>(
+      q_blk, k_blk, frame_idx, block_idx, block_score, D);
+  return cuda_status(cudaGetLastError());
+}
+
+size_t attn_ws_bytes(const Dims& D) {
+  const size_t nt = (size_t)lf::tile_count(D) * D.H;
+  return align_up(nt * lf::plan_stride(D) * sizeof(uint32_t), 256) +
+         align_up(nt * sizeof(int32_t), 256);
+}
+
+template <int HD, int BLK>
+int launch_attn_t(const Dims& D, lf::AttnParams& p, cudaStream_t st) {
+  using L = lf::AttnLayout<HD>;
+  auto kern = lf::attn_kernel<HD, BLK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return LF_ERR_CUDA;
+  dim3 grid(lf::tile_count(D), D.H);
+  kern<<<grid, lf::kAttnThreads, L::kAlloc, st>>>(p, D);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_cur,
+                const void* k_cache, const void* v_cache, const int32_t* hist_slots,
+                const int32_t* sink_slots, const int32_t* block_idx, void* out, float* lse,
+                void* workspace, cudaStream_t st) {
+  const size_t nt = (size_t)lf::tile_count(D) * D.H;
+  uint32_t* plan = static_cast<uint32_t*>(workspace);
+  int32_t* plan_cnt = reinterpret_cast<int32_t*>(
+      static_cast<uint8_t*>(workspace) + align_up(nt * lf::plan_stride(D) * sizeof(uint32_t), 256));
+  lf::plan_kernel<<<dim3(lf::tile_count(D), D.H), 32, 0, st>>>(
+      D.F > 0 ? block_idx : nullptr, plan, plan_cnt, D);
+  int rc = cuda_status(cudaGetLastError());
+  if (rc != LF_OK) return rc;
+
+  lf::AttnParams p;
+  memset(&p, 0, sizeof(p));
+  const int HD = D.H * D.d;
+  if ((rc = encode_rows(&p.tm_q, q, HD, D.ncur, 0)) != LF_OK) return rc;
+  if ((rc = encode_rows(&p.tm_kc, k_cur, HD, D.ncur, 0)) != LF_OK) return rc;
+  if ((rc = encode_rows(&p.tm_vc, v_cur, HD, D.ncur, 0)) != LF_OK) return rc;
+  if (D.F + D.S > 0) {
+    if ((rc = encode_rows(&p.tm_kh, k_cache, HD, D.T, D.n_slots)) != LF_OK) return rc;
+    if ((rc = encode_rows(&p.tm_vh, v_cache, HD, D.T, D.n_slots)) != LF_OK) return rc;
+  } else {   // no cache frames: the maps are never used; point them at the current chunk
+    p.tm_kh = p.tm_kc;
+    p.tm_vh = p.tm_vc;
+  }
+  p.plan = plan;
+  p.plan_cnt = plan_cnt;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  for (int i = 0; i < D.S; ++i) p.slots[i] = sink_slots[i];
+  for (int i = 0; i < D.F; ++i) p.slots[D.S + i] = hist_slots[i];
+  if (D.d == 128) return D.B == 64 ? launch_attn_t<128, 64>(D, p, st) : launch_attn_t<128, 128>(D, p, st);
+  return D.B == 64 ? launch_attn_t<64, 64>(D, p, st) : launch_attn_t<64, 128>(D, p, st);
+}
+
+// forward workspace carve-up
+struct FwdWs {
+  float *q_blk, *k_blk, *k_frm;
+  int32_t *frame_idx, *block_idx;
+  void* attn;
+  size_t bytes;
+};
+
+FwdWs carve(const Dims& D, void* base) {
+  FwdWs w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t n) { uint8_t* r = p ? p + off : nullptr; off += align_up(n, 256); return r; };
+  w.q_blk = reinterpret_cast<float*>(take((size_t)D.H * D.nqb * D.d * 4));
+  w.k_blk = reinterpret_cast<float*>(take((size_t)D.H * D.F * D.nbpf * D.d * 4));
+  w.k_frm = reinterpret_cast<float*>(take((size_t)D.H * D.F * D.d * 4));
+  w.frame_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.kf * 4));
+  w.block_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.nsel * 4));
+  w.attn = take(attn_ws_bytes(D));
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+extern "C" {
+
+int lf_abi_version(void) { return LF_ABI_VERSION; }
+
+const char* lf_status_string(int s) {
+  switch (s) {
+    case LF_OK: return "ok";
+    case LF_ERR_INVALID_ARG: return "invalid argument";
+    case LF_ERR_UNSUPPORTED: return "unsupported shape";
+    case LF_ERR_CUDA: return "CUDA error";
+    case LF_ERR_TIMEOUT: return "device wait timed out";
+    case LF_ERR_WORKSPACE: return "workspace missing or too small";
+    case LF_ERR_BAD_INDEX: return "index out of range in a device list";
+    default: return "unknown status";
+  }
+}
+
+int lf_compress(const lf_shape* shape, const void* q, const void* k_cache,
+                const int32_t* hist_slots, float* q_blk, float* k_blk, float* k_frm,
+                cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (q == nullptr || q_blk == nullptr || !aligned(q, 16) || !aligned(q_blk, 16))
+    return LF_ERR_INVALID_ARG;
+  if (D.F > 0) {
+    if (k_cache == nullptr || k_blk == nullptr || k_frm == nullptr || !aligned(k_cache, 16) ||
+        !aligned(k_blk, 16) || !aligned(k_frm, 16))
+      return LF_ERR_INVALID_ARG;
+    if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
+  }
+  return launch_compress(D, q, k_cache, hist_slots, q_blk, k_blk, k_frm, stream);
+}
+
+int lf_select_frames(const lf_shape* shape, const float* q_blk, const float* k_frm,
+                     int32_t* frame_idx, float* frame_score, cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (D.F < 1) return LF_ERR_INVALID_ARG;
+  if (q_blk == nullptr || k_frm == nullptr || frame_idx == nullptr || !aligned(q_blk, 16) ||
+      !aligned(k_frm, 16) || !aligned(frame_idx, 4) || (frame_score && !aligned(frame_score, 4)))
+    return LF_ERR_INVALID_ARG;
+  return launch_select_frames(D, q_blk, k_frm, frame_idx, frame_score, stream);
+}
+
+int lf_select_blocks(const lf_shape* shape, const float* q_blk, const float* k_blk,
+                     const int32_t* frame_idx, int32_t* block_idx, float* block_score,
+                     cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (D.F < 1) return LF_ERR_INVALID_ARG;
+  if (q_blk == nullptr || k_blk == nullptr || frame_idx == nullptr || block_idx == nullptr ||
+      !aligned(q_blk, 16) || !aligned(k_blk, 16) || !aligned(frame_idx, 4) ||
+      !aligned(block_idx, 4) || (block_score && !aligned(block_score, 4)))
+    return LF_ERR_INVALID_ARG;
+  return launch_select_blocks(D, q_blk, k_blk, frame_idx, block_idx, block_score, stream);
+}
+
+size_t lf_attn_workspace_size(const lf_shape* shape) {
+  Dims D;
+  if (make_dims(shape, &D) != LF_OK) return 0;
+  return attn_ws_bytes(D);
+}
+
+int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur,
+                         const void* v_cur, const void* k_cache, const void* v_cache,
+                         const int32_t* hist_slots, const int32_t* sink_slots,
+                         const int32_t* block_idx, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (q == nullptr || k_cur == nullptr || v_cur == nullptr || out == nullptr ||
+      !aligned(q, 16) || !aligned(k_cur, 16) || !aligned(v_cur, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)))
+    return LF_ERR_INVALID_ARG;
+  if (D.F + D.S > 0 && (k_cache == nullptr || v_cache == nullptr || !aligned(k_cache, 16) ||
+                        !aligned(v_cache, 16)))
+    return LF_ERR_INVALID_ARG;
+  if (D.F > 0 && (block_idx == nullptr || !aligned(block_idx, 4))) return LF_ERR_INVALID_ARG;
+  if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
+  if ((rc = check_slots(sink_slots, D.S, D.n_slots)) != LF_OK) return rc;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < attn_ws_bytes(D))
+    return LF_ERR_WORKSPACE;
+  return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, block_idx,
+                     out, lse, workspace, stream);
+}
+
+size_t lf_forward_workspace_size(const lf_shape* shape) {
+  Dims D;
+  if (make_dims(shape, &D) != LF_OK) return 0;
+  return carve(D, nullptr).bytes;
+}
+
+int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
+                     const void* v_cur, const void* k_cache, const void* v_cache,
+                     const int32_t* hist_slots, const int32_t* sink_slots,
+                     void* workspace, size_t workspace_bytes, void* out, float* lse,
+                     int32_t* block_idx_out, cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (q == nullptr || k_cur == nullptr || v_cur == nullptr || out == nullptr ||
+      !aligned(q, 16) || !aligned(k_cur, 16) || !aligned(v_cur, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)) || (block_idx_out && !aligned(block_idx_out, 4)))
+    return LF_ERR_INVALID_ARG;
+  if (D.F + D.S > 0 && (k_cache == nullptr || v_cache == nullptr || !aligned(k_cache, 16) ||
+                        !aligned(v_cache, 16)))
+    return LF_ERR_INVALID_ARG;
+  if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
+  if ((rc = check_slots(sink_slots, D.S, D.n_slots)) != LF_OK) return rc;
+  const FwdWs need = carve(D, nullptr);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need.bytes)
+    return LF_ERR_WORKSPACE;
+  const FwdWs w = carve(D, workspace);
+  int32_t* bidx = block_idx_out ? block_idx_out : w.block_idx;
+  if (D.F > 0) {
+    if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, w.k_frm, stream)) != LF_OK)
+      return rc;
+    if ((rc = launch_select_frames(D, w.q_blk, w.k_frm, w.frame_idx, nullptr, stream)) != LF_OK)
+      return rc;
+    if ((rc = launch_select_blocks(D, w.q_blk, w.k_blk, w.frame_idx, bidx, nullptr, stream)) != LF_OK)
+      return rc;
+  }
+  return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, bidx, out,
+                     lse, w.attn, stream);
+}
+
+int lf_device_status(int reset) {
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LF_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, lf::g_lf_status, sizeof(int)) != cudaSuccess) return LF_ERR_CUDA;
+  if (reset && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(lf::g_lf_status, &zero, sizeof(int)) != cudaSuccess) return LF_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

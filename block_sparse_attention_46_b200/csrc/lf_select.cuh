@@ -1,0 +1,286 @@
+// lf_select.cuh — stages (a)-(c) of hierarchical sparse attention: token compression
+// (mean pooling of query and key blocks, frame pooling) and the two-stage top-k
+// selection of history frames and blocks.
+//
+// [LF-gist 2.2] "Light Forcing: Accelerating Autoregressive Video Diffusion via Sparse
+// Attention" (gist.science explainer), section 2.2: queries and keys are compressed by
+// mean pooling at block and frame granularity; each query block first retrieves a few
+// history frames with the frame-level compressed keys, then the important blocks inside
+// those frames with the block-level compressed keys.
+// [LF-yly 三] the youleyou article, section 三: the same stages; similarity is an inner
+// product.
+#pragma once
+#include "lf_common.cuh"
+
+namespace lf {
+
+// ---------------------------------------------------------------------------------
+// (a) Pooling.  One CTA row (blockIdx.x) is one block of tokens: the first nqb rows are
+// the current chunk's query blocks, the next F*nbpf rows the history key blocks.  Each
+// thread owns 8 consecutive channels of the H*d-wide token row (one 16-byte load per
+// token), so a warp reads 512 contiguous bytes per token.  Sums are fp32, token order.
+// ---------------------------------------------------------------------------------
+struct PoolArgs {
+  const __nv_bfloat16* q;        // [ncur, H, d]
+  const __nv_bfloat16* k_cache;  // [n_slots, T, H, d]
+  float* q_blk;                  // [H, nqb, d]
+  float* k_blk;                  // [H, F, nbpf, d]
+  int hist_slots[LF_MAX_FRAMES];
+};
+
+constexpr int kPoolThreads = 64;
+constexpr int kPoolUnroll = 8;
+
+__global__ void __launch_bounds__(kPoolThreads)
+pool_blocks_kernel(const __grid_constant__ PoolArgs a, const Dims D) {
+  const int unit = blockIdx.x;
+  const int HD = D.H * D.d;
+  const int vec = blockIdx.y * kPoolThreads + threadIdx.x;   // 8-channel group
+  if (vec * 8 >= HD) return;
+
+  const __nv_bfloat16* base;
+  int ntok;
+  float* dst;
+  const int h = (vec * 8) / D.d, c0 = (vec * 8) % D.d;
+  if (unit < D.nqb) {
+    const int f = unit / D.nbpf, b = unit % D.nbpf;
+    ntok = block_len(D, b);
+    base = a.q + ((size_t)f * D.T + (size_t)b * D.B) * HD;
+    dst = a.q_blk + ((size_t)h * D.nqb + unit) * D.d + c0;
+  } else {
+    const int u = unit - D.nqb;
+    const int f = u / D.nbpf, b = u % D.nbpf;
+    const int slot = a.hist_slots[f];
+    ntok = block_len(D, b);
+    base = a.k_cache + ((size_t)slot * D.T + (size_t)b * D.B) * HD;
+    dst = a.k_blk + (((size_t)h * D.F + f) * D.nbpf + b) * D.d + c0;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(base) + vec;
+  const size_t stride = HD / 8;     // uint4 per token row
+
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+
+  int t = 0;
+  for (; t + kPoolUnroll <= ntok; t += kPoolUnroll) {
+    uint4 v[kPoolUnroll];
+#pragma unroll
+    for (int u = 0; u < kPoolUnroll; ++u) v[u] = __ldg(src + (size_t)(t + u) * stride);
+#pragma unroll
+    for (int u = 0; u < kPoolUnroll; ++u) {
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 f2 = __bfloat1622float2(p[i]);
+        acc[2 * i] += f2.x;
+        acc[2 * i + 1] += f2.y;
+      }
+    }
+  }
+  for (; t < ntok; ++t) {
+    uint4 v = __ldg(src + (size_t)t * stride);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f2 = __bfloat1622float2(p[i]);
+      acc[2 * i] += f2.x;
+      acc[2 * i + 1] += f2.y;
+    }
+  }
+  const float inv = 1.0f / (float)ntok;
+  float4* o = reinterpret_cast<float4*>(dst);
+  o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+}
+
+// Frame pooling from the block means: k_frm = sum_b len_b * k_blk[b] / T (the frame mean
+// over all T tokens, since block sums are len_b * mean_b).  One thread per channel.
+__global__ void pool_frames_kernel(const float* __restrict__ k_blk, float* __restrict__ k_frm,
+                                   const Dims D) {
+  const int f = blockIdx.x, h = blockIdx.y;
+  const float* src = k_blk + ((size_t)h * D.F + f) * D.nbpf * D.d;
+  const float invT = 1.0f / (float)D.T;
+  for (int c = threadIdx.x; c < D.d; c += blockDim.x) {
+    float s = 0.f;
+    for (int b = 0; b < D.nbpf; ++b) s += (float)block_len(D, b) * src[(size_t)b * D.d + c];
+    k_frm[((size_t)h * D.F + f) * D.d + c] = s * invT;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Warp top-k helpers.  Order: larger score first; equal scores -> lower index first.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ bool better(float s1, int i1, float s2, int i2) {
+  return s1 > s2 || (s1 == s2 && i1 < i2);
+}
+
+// Warp-wide argmax of (score, index) pairs with the order above; every lane gets it.
+__device__ __forceinline__ void warp_argmax(float& s, int& i) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    float so = __shfl_xor_sync(0xffffffffu, s, off);
+    int io = __shfl_xor_sync(0xffffffffu, i, off);
+    if (better(so, io, s, i)) { s = so; i = io; }
+  }
+}
+
+constexpr int kMaxPerLane = 8;   // candidates per lane: up to 256 frames or blocks
+
+// Selects the k best of n candidates held lane-strided (candidate c = lane + 32*j lives
+// in sc[j] of lane c%32).  Returns in `taken` (bit j per lane) the chosen candidates.
+__device__ __forceinline__ uint32_t warp_topk(const float* sc, int n, int k) {
+  const int lane = threadIdx.x & 31;
+  uint32_t taken = 0;
+  for (int r = 0; r < k; ++r) {
+    float bs = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < kMaxPerLane; ++j) {
+      const int c = lane + 32 * j;
+      if (c < n && !((taken >> j) & 1u) && better(sc[j], c, bs, bi)) { bs = sc[j]; bi = c; }
+    }
+    warp_argmax(bs, bi);
+    if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+  }
+  return taken;
+}
+
+// Writes the chosen candidate ids ascending: out[pos] = id_base + c.
+__device__ __forceinline__ void warp_write_ascending(uint32_t taken, int n, int32_t* out,
+                                                     int id_base) {
+  const int lane = threadIdx.x & 31;
+  int before = 0;
+#pragma unroll
+  for (int j = 0; j < kMaxPerLane; ++j) {
+    if (32 * j >= n) break;
+    const uint32_t m = __ballot_sync(0xffffffffu, (taken >> j) & 1u);
+    if ((taken >> j) & 1u) out[before + __popc(m & ((1u << lane) - 1u))] = id_base + lane + 32 * j;
+    before += __popc(m);
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// (b) Frame selection.  CTA = (group of 8 query blocks, head); k_frm[h] is staged in shared
+// memory with a padded row pitch; warp w takes query block 8*blockIdx.x + w, lane c scores
+// frames c, c+32, ... with a full-length dot product in fixed order.
+// ---------------------------------------------------------------------------------
+constexpr int kSelWarps = 8;
+
+__global__ void __launch_bounds__(kSelWarps * 32)
+select_frames_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_frm,
+                     int32_t* __restrict__ frame_idx, float* __restrict__ frame_score,
+                     const Dims D) {
+  extern __shared__ float4 sm4[];
+  float* sk = reinterpret_cast<float*>(sm4);
+  const int h = blockIdx.y;
+  const int pitch = D.d + 4;
+  float* sq = sk + (size_t)D.F * pitch;               // [kSelWarps][d]
+  for (int i = threadIdx.x; i < D.F * (D.d / 4); i += blockDim.x) {
+    const int f = i / (D.d / 4), c4 = i % (D.d / 4);
+    reinterpret_cast<float4*>(sk + (size_t)f * pitch)[c4] =
+        reinterpret_cast<const float4*>(k_frm + ((size_t)h * D.F + f) * D.d)[c4];
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = blockIdx.x * kSelWarps + warp;
+  if (qb < D.nqb)
+    for (int c4 = lane; c4 < D.d / 4; c4 += 32)
+      reinterpret_cast<float4*>(sq + warp * D.d)[c4] =
+          reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + qb) * D.d)[c4];
+  __syncthreads();
+  if (qb >= D.nqb) return;
+
+  float sc[kMaxPerLane];
+  const float* qv = sq + warp * D.d;
+#pragma unroll
+  for (int j = 0; j < kMaxPerLane; ++j) {
+    const int f = lane + 32 * j;
+    float s = -INFINITY;
+    if (f < D.F) {
+      const float* kv = sk + (size_t)f * pitch;
+      s = 0.f;
+      for (int c = 0; c < D.d; c += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(qv + c);
+        const float4 b = *reinterpret_cast<const float4*>(kv + c);
+        s = fmaf(a.x, b.x, s); s = fmaf(a.y, b.y, s); s = fmaf(a.z, b.z, s); s = fmaf(a.w, b.w, s);
+      }
+      if (frame_score) frame_score[((size_t)h * D.nqb + qb) * D.F + f] = s;
+    }
+    sc[j] = s;
+  }
+  const uint32_t taken = warp_topk(sc, D.F, D.kf);
+  warp_write_ascending(taken, D.F, frame_idx + ((size_t)h * D.nqb + qb) * D.kf, 0);
+}
+
+// ---------------------------------------------------------------------------------
+// (c) Block selection inside chosen frames.  CTA = (history frame f, head h): k_blk[h, f]
+// is staged in shared memory once; each warp walks the query blocks of head h whose
+// chosen-frame list holds f (at rank j), scores the frame's blocks (lane c: blocks c,
+// c+32, ...), keeps the kb best and writes them, ascending, to slots [j*kb, (j+1)*kb) of
+// block_idx[h, qb] — ascending overall because the frame list is ascending.
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kSelWarps * 32)
+select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_blk,
+                     const int32_t* __restrict__ frame_idx, int32_t* __restrict__ block_idx,
+                     float* __restrict__ block_score, const Dims D) {
+  extern __shared__ float4 sm4[];
+  float* sk = reinterpret_cast<float*>(sm4);
+  const int f = blockIdx.x, h = blockIdx.y;
+  const int pitch = D.d + 4;
+  float* sq = sk + (size_t)D.nbpf * pitch;            // [kSelWarps][d]
+  for (int i = threadIdx.x; i < D.nbpf * (D.d / 4); i += blockDim.x) {
+    const int b = i / (D.d / 4), c4 = i % (D.d / 4);
+    reinterpret_cast<float4*>(sk + (size_t)b * pitch)[c4] =
+        reinterpret_cast<const float4*>(k_blk + (((size_t)h * D.F + f) * D.nbpf + b) * D.d)[c4];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* qv = sq + warp * D.d;
+  for (int qb = warp; qb < D.nqb; qb += kSelWarps) {
+    const int32_t* fl = frame_idx + ((size_t)h * D.nqb + qb) * D.kf;
+    // rank of f in the (ascending) chosen list; validate the list on the way
+    int rank = -1;
+    bool bad = false;
+    for (int j = lane; j < D.kf; j += 32) {
+      const int v = fl[j];
+      if (v < 0 || v >= D.F || (j > 0 && fl[j - 1] >= v)) bad = true;
+      if (v == f) rank = j;
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    rank = __reduce_max_sync(0xffffffffu, rank);
+    if (bad) {
+      if (lane == 0 && f == 0) record_status(LF_ERR_BAD_INDEX);
+      continue;
+    }
+    if (rank < 0) continue;
+    for (int c4 = lane; c4 < D.d / 4; c4 += 32)
+      reinterpret_cast<float4*>(qv)[c4] =
+          reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + qb) * D.d)[c4];
+    __syncwarp();
+    float sc[kMaxPerLane];
+#pragma unroll
+    for (int j = 0; j < kMaxPerLane; ++j) {
+      const int b = lane + 32 * j;
+      float s = -INFINITY;
+      if (b < D.nbpf) {
+        const float* kv = sk + (size_t)b * pitch;
+        s = 0.f;
+        for (int c = 0; c < D.d; c += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(qv + c);
+          const float4 y = *reinterpret_cast<const float4*>(kv + c);
+          s = fmaf(x.x, y.x, s); s = fmaf(x.y, y.y, s); s = fmaf(x.z, y.z, s); s = fmaf(x.w, y.w, s);
+        }
+        if (block_score)
+          block_score[(((size_t)h * D.nqb + qb) * D.kf + rank) * D.nbpf + b] = s;
+      }
+      sc[j] = s;
+    }
+    const uint32_t taken = warp_topk(sc, D.nbpf, D.kb);
+    warp_write_ascending(taken, D.nbpf,
+                         block_idx + ((size_t)h * D.nqb + qb) * D.nsel + (size_t)rank * D.kb,
+                         f * D.nbpf);
+    __syncwarp();
+  }
+}
+
+}  // namespace lf

@@ -1,0 +1,163 @@
+/*
+ * lf.h — C ABI of liblf, a B200 (sm_100a) implementation of Light Forcing's hierarchical
+ * sparse attention (HSA) for chunk-wise autoregressive video diffusion.
+ *
+ * The method (sources named by page title and section):
+ *   [LF-gist] "Light Forcing: Accelerating Autoregressive Video Diffusion via Sparse
+ *             Attention" (gist.science explainer), section 2.2 Hierarchical Sparse
+ *             Attention — token compression by mean pooling per block and per frame,
+ *             two-stage mask selection (frames, then blocks inside chosen frames),
+ *             attention only on the chosen frame-block pairs.
+ *   [LF-yly]  "南洋理工大学AI新突破 视频生成引擎模仿人脑高效学习" (m.youleyou.com),
+ *             section 三 — the same three stages; frames retrieved by inner products.
+ *   [SF]      Self Forcing article, rolling KV cache paragraph — cache of the last L
+ *             frames, oldest evicted first.
+ *   [RF]      "南洋理工大学突破：AI实现实时流式视频生成" (163.com, Rolling Forcing),
+ *             section 三 — first frames kept as permanent anchors (sink frames).
+ *
+ * One call of the attention layer = (a) lf_compress, (b) lf_select_frames,
+ * (c) lf_select_blocks, (d) lf_block_sparse_attn; lf_forward_chunk chains all four.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Tensors.  bf16 tensors are token-major [tokens, H, d], contiguous:
+ *      q, k_cur, v_cur   : [n_cur_frames*T, H, d]  (the current chunk, raster order)
+ *      k_cache, v_cache  : [n_slots, T, H, d]      (one latent frame per slot)
+ *      out               : [n_cur_frames*T, H, d]
+ *    Pooled and score tensors are fp32, index tensors int32, all contiguous:
+ *      q_blk  [H, n_qb, d]           k_blk [H, n_hist, n_bpf, d]    k_frm [H, n_hist, d]
+ *      frame_idx [H, n_qb, kf]       block_idx [H, n_qb, kf*kb]      lse [H, n_cur_frames*T]
+ *    with T = tokens_per_frame, B = block, n_bpf = ceil(T/B), n_qb = n_cur_frames*n_bpf,
+ *    kf = min(k_f, n_hist), kb = min(k_b, n_bpf).
+ *  Blocks.  Block b of a frame covers tokens [b*B, min((b+1)*B, T)); the last block of a
+ *    frame is shorter when B does not divide T.  Query block qb = frame*n_bpf + b.
+ *    A global history block id is g = f*n_bpf + b, f being the history position.
+ *  Frame lists.  hist_slots[n_hist] and sink_slots[n_sink] are HOST int32 arrays giving
+ *    the cache slot of each history / sink frame, oldest first; they are read during
+ *    the call only.  Rolling the cache means rewriting slot ids; nothing is copied.
+ *  Memory.  Every other pointer is caller-owned DEVICE memory on the current device.
+ *    The library never allocates or frees.  bf16 tensors and fp32 tensors must be
+ *    16-byte aligned; int32 tensors 4-byte aligned.
+ *  Streams.  Work is enqueued on `stream` and is asynchronous; a return of LF_OK means
+ *    the arguments were valid and the launches were accepted.  Device-detected errors
+ *    (an index out of range in a caller-supplied list, a device wait that ran out of
+ *    time) are recorded in a per-device status word read by lf_device_status().
+ *  Validation.  Every argument check happens before the first launch; on error nothing
+ *    is enqueued.
+ *  Determinism.  Identical inputs give bit-identical outputs (no float atomics).
+ */
+#ifndef LF_H_
+#define LF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LF_ABI_VERSION 1
+
+/* status codes */
+#define LF_OK               0
+#define LF_ERR_INVALID_ARG  1   /* null/misaligned pointer, inconsistent sizes          */
+#define LF_ERR_UNSUPPORTED  2   /* d or block outside {64,128}, or a size limit exceeded */
+#define LF_ERR_CUDA         3   /* a CUDA runtime or launch error                        */
+#define LF_ERR_TIMEOUT      4   /* a bounded device wait expired (from lf_device_status) */
+#define LF_ERR_WORKSPACE    5   /* workspace pointer null or smaller than required       */
+#define LF_ERR_BAD_INDEX    6   /* device found an index out of range (lf_device_status) */
+
+/* size limits checked by every entry point */
+#define LF_MAX_FRAMES       256     /* n_sink + n_hist                                  */
+#define LF_MAX_T            16384   /* tokens per frame                                 */
+#define LF_MAX_SELECTED     1024    /* kf * kb per query block                          */
+
+typedef struct lf_shape {
+    int32_t H;                /* heads, >= 1                                              */
+    int32_t d;                /* head dimension: 64 or 128                                */
+    int32_t tokens_per_frame; /* T, 1..LF_MAX_T                                           */
+    int32_t block;            /* B, block size in tokens: 64 or 128                       */
+    int32_t n_cur_frames;     /* F_c, frames in the current chunk, >= 1                   */
+    int32_t n_hist;           /* F, selectable history frames, >= 0                       */
+    int32_t n_sink;           /* S_k, always-dense sink frames, >= 0                      */
+    int32_t n_slots;          /* frames the cache tensors hold; slot ids are < n_slots    */
+    int32_t k_f;              /* frames kept per query block (>= 1 when n_hist > 0)       */
+    int32_t k_b;              /* blocks kept per chosen frame (>= 1 when n_hist > 0)      */
+    float   scale;            /* softmax scale applied to q.k, normally 1/sqrt(d)         */
+} lf_shape;
+
+/* (a) Token compression [LF-gist 2.2 "token compression"; LF-yly 三, first stage].
+ * q_blk[h, qb]   = mean of the query tokens of block qb of the current chunk;
+ * k_blk[h, f, b] = mean of the keys of block b of history frame f;
+ * k_frm[h, f]    = mean of all T keys of history frame f.
+ * Accumulation is fp32 in a fixed order.  With n_hist == 0 only q_blk is written and
+ * k_cache / k_blk / k_frm may be NULL. */
+int lf_compress(const lf_shape* shape, const void* q, const void* k_cache,
+                const int32_t* hist_slots, float* q_blk, float* k_blk, float* k_frm,
+                cudaStream_t stream);
+
+/* (b) Frame-level selection [LF-gist 2.2, mask selection step 1; LF-yly 三].
+ * score[h, qb, f] = q_blk[h, qb] . k_frm[h, f]; frame_idx[h, qb] = the kf frames with the
+ * largest scores, ties to the lower index, written in ascending order.
+ * frame_score (nullable) receives all scores [H, n_qb, n_hist].  Requires n_hist >= 1. */
+int lf_select_frames(const lf_shape* shape, const float* q_blk, const float* k_frm,
+                     int32_t* frame_idx, float* frame_score, cudaStream_t stream);
+
+/* (c) Block-level selection inside the chosen frames [LF-gist 2.2, mask selection step 2].
+ * For each chosen frame f of (h, qb): score[b] = q_blk[h, qb] . k_blk[h, f, b]; keep the
+ * kb largest (ties to the lower index).  block_idx[h, qb] lists the kf*kb global block
+ * ids g = f*n_bpf + b in ascending order.  block_score (nullable) receives the scores of
+ * the chosen frames [H, n_qb, kf, n_bpf].  frame_idx entries must be ascending and
+ * < n_hist (violations are recorded as LF_ERR_BAD_INDEX and the entry is skipped). */
+int lf_select_blocks(const lf_shape* shape, const float* q_blk, const float* k_blk,
+                     const int32_t* frame_idx, int32_t* block_idx, float* block_score,
+                     cudaStream_t stream);
+
+/* Workspace bytes lf_block_sparse_attn needs for this shape (its per-tile key plans). */
+size_t lf_attn_workspace_size(const lf_shape* shape);
+
+/* (d) Block-sparse attention [LF-gist 2.2 "execution"; LF-yly 三, last stage].
+ * For every query token of query block qb and head h, one joint softmax over
+ *   - every key of the current chunk (k_cur, dense, no causal mask),
+ *   - every key of every sink frame (k_cache at sink_slots) [RF],
+ *   - the keys of the history blocks listed in block_idx[h, qb] (k_cache at hist_slots)
+ * of scale * q.k, applied to the matching values.  out receives bf16; lse (nullable)
+ * receives the natural-log normaliser log(sum exp(scale*q.k)) in fp32.
+ * block_idx: [H, n_qb, kf*kb] ascending global ids (ignored, may be NULL, when
+ * n_hist == 0).  Ids out of range or not ascending are recorded as LF_ERR_BAD_INDEX and
+ * dropped.  Compute: tcgen05 bf16 MMAs with fp32 accumulation in tensor memory, fp32
+ * online softmax. */
+int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur,
+                         const void* v_cur, const void* k_cache, const void* v_cache,
+                         const int32_t* hist_slots, const int32_t* sink_slots,
+                         const int32_t* block_idx, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes lf_forward_chunk needs: pooled tensors, index lists and key plans. */
+size_t lf_forward_workspace_size(const lf_shape* shape);
+
+/* (a)->(b)->(c)->(d) in one call.  block_idx_out (nullable) receives the selected block
+ * ids [H, n_qb, kf*kb]; lse is nullable.  With n_hist == 0 no selection runs and the
+ * attention covers the current chunk and the sink frames. */
+int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
+                     const void* v_cur, const void* k_cache, const void* v_cache,
+                     const int32_t* hist_slots, const int32_t* sink_slots,
+                     void* workspace, size_t workspace_bytes, void* out, float* lse,
+                     int32_t* block_idx_out, cudaStream_t stream);
+
+/* Reads (synchronising the current device) and optionally clears the device status word
+ * of the current device: LF_OK, LF_ERR_BAD_INDEX or LF_ERR_TIMEOUT.  Returns LF_ERR_CUDA
+ * if the read itself fails. */
+int lf_device_status(int reset);
+
+/* Static text for a status code. */
+const char* lf_status_string(int status);
+
+/* LF_ABI_VERSION of the loaded library. */
+int lf_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LF_H_ */

@@ -1,0 +1,97 @@
+"""The C ABI without a GPU: the library loads, exports every symbol include/lf.h declares,
+and rejects invalid arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_46_b200 as lf
+import lf_workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "lf.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(lf_\w+)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_46_b200 import build
+    build.build()
+    return lf.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "lf_forward_chunk" in names and "lf_block_sparse_attn" in names
+    raw = ctypes.CDLL(lf.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    assert lf.lf_abi_version() == 1
+
+
+def _shape(**kw):
+    base = dict(H=2, d=64, T=256, block=64, n_cur_frames=1, n_hist=4, n_sink=0, n_slots=4,
+                k_f=2, k_b=2, scale=0.125)
+    base.update(kw)
+    return W.Shape(**base)
+
+
+FAKE = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
+
+
+def _attn(lib, shape, hist=(0, 1, 2, 3), sinks=(), ws=1 << 20, wsptr=FAKE, bidx=FAKE):
+    sh = lf.make_shape(shape)
+    h = (ctypes.c_int32 * max(len(hist), 1))(*hist)
+    s = (ctypes.c_int32 * max(len(sinks), 1))(*sinks)
+    return lib.lf_block_sparse_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE,
+                                     ctypes.cast(h, ctypes.POINTER(ctypes.c_int32)),
+                                     ctypes.cast(s, ctypes.POINTER(ctypes.c_int32)), bidx, FAKE,
+                                     None, wsptr, ws, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(d=256), 2), (dict(block=32), 2), (dict(H=0), 1),
+    (dict(n_cur_frames=0), 1), (dict(T=0), 1), (dict(T=20000), 2), (dict(n_hist=-1), 1),
+    (dict(k_f=0), 1), (dict(k_b=0), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(n_hist=300, n_slots=300), 2),
+])
+def test_shape_validation(lib, kw, code):
+    assert _attn(lib, _shape(**kw), hist=tuple(range(min(kw.get("n_hist", 4), 256)))
+                 if kw.get("n_hist", 4) > 0 else ()) == code
+
+
+def test_slot_and_workspace_validation(lib):
+    assert _attn(lib, _shape(), hist=(0, 1, 2, 4)) == 1                # slot >= n_slots
+    assert _attn(lib, _shape(), hist=(0, 1, -1, 2)) == 1
+    assert _attn(lib, _shape(n_sink=1, n_slots=5), hist=(0, 1, 2, 3), sinks=(9,)) == 1
+    assert _attn(lib, _shape(), ws=16) == 5                            # workspace too small
+    assert _attn(lib, _shape(), wsptr=None) == 5
+    assert _attn(lib, _shape(), bidx=None) == 1                        # needs block_idx
+
+
+def test_misaligned_pointer_rejected(lib):
+    sh = lf.make_shape(_shape())
+    h = (ctypes.c_int32 * 4)(0, 1, 2, 3)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    rc = lib.lf_compress(ctypes.byref(sh), odd, FAKE, ctypes.cast(h, ctypes.POINTER(ctypes.c_int32)),
+                         FAKE, FAKE, FAKE, None)
+    assert rc == 1
+
+
+def test_workspace_sizes(lib):
+    s480 = W.p480_shape()
+    attn = lf.lf_attn_workspace_size(s480)
+    fwd = lf.lf_forward_workspace_size(s480)
+    # 38 tiles x 12 heads x (2 x 72) plan entries + counts, and the pooled tensors
+    assert attn >= 38 * 12 * 144 * 4
+    assert fwd >= attn + 12 * 18 * 25 * 128 * 4
+    assert lf.lf_attn_workspace_size(_shape(d=96)) == 0
+
+
+def test_status_strings(lib):
+    assert lf.lf_status_string(0) == "ok"
+    assert "timed out" in lf.lf_status_string(4)

@@ -1,0 +1,191 @@
+"""CUDA path (through the C ABI) against the float64 oracle on the same seeded inputs.
+
+Small shapes are compared element by element for every stage; they span several query
+and key tiles, ragged frame tails (T not a multiple of B, T < B), odd query-block counts
+(a tile with one query block), sinks, no history, and k_f / k_b at or above their
+limits.  The full-size workloads (the 480p chunk the benchmark times, the large-model
+stress, a rolling-cache chunk and a growth-sweep chunk) run the exact benchmark call and
+are checked on all selected indices and on sampled query blocks of the output, plus
+properties that hold at any size (every row written and finite).
+"""
+import numpy as np
+import pytest
+import torch
+
+import lf_workloads as W
+from oracle import hsa64 as O
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": lambda: W.tiny(0),
+    "ragged_d64": lambda: W.random_small(1, H=2, d=64, T=200, block=64, n_cur_frames=1,
+                                         n_hist=5, n_sink=0, k_f=2, k_b=2),
+    "sinks_d128": lambda: W.random_small(2, H=2, d=128, T=200, block=64, n_cur_frames=3,
+                                         n_hist=4, n_sink=1, k_f=3, k_b=2),
+    "b128": lambda: W.random_small(3, H=3, d=128, T=300, block=128, n_cur_frames=2,
+                                   n_hist=3, n_sink=0, k_f=2, k_b=2),
+    "k_at_limits": lambda: W.random_small(4, H=2, d=64, T=130, block=128, n_cur_frames=1,
+                                          n_hist=2, n_sink=2, k_f=5, k_b=9),
+    "T_below_B_odd_tiles": lambda: W.random_small(5, H=1, d=128, T=40, block=64,
+                                                  n_cur_frames=3, n_hist=6, n_sink=0,
+                                                  k_f=3, k_b=1),
+    "no_history": lambda: W.random_small(6, H=2, d=128, T=192, block=64, n_cur_frames=1,
+                                         n_hist=0, n_sink=0, k_f=1, k_b=1),
+    "sinks_only": lambda: W.random_small(7, H=2, d=64, T=160, block=64, n_cur_frames=2,
+                                         n_hist=0, n_sink=3, k_f=1, k_b=1),
+    "frames_1560_b64": lambda: W.random_small(8, H=2, d=128, T=1560, block=64,
+                                              n_cur_frames=1, n_hist=3, n_sink=1,
+                                              k_f=2, k_b=12),
+    "frames_1560_b128": lambda: W.random_small(9, H=2, d=128, T=1560, block=128,
+                                               n_cur_frames=1, n_hist=4, n_sink=0,
+                                               k_f=2, k_b=5),
+}
+
+
+def _oracle_selection(ci):
+    sh = ci.shape
+    qb = O.compress_queries(ci.q, sh.T, sh.block)
+    kb, kf = O.compress_keys(ci.k_cache, ci.hist_slots, sh.T, sh.block)
+    fidx, sf = O.select_frames(qb, kf, sh.k_f)
+    bidx, sb = O.select_blocks(qb, kb, fidx, sh.k_b)
+    return qb, kb, kf, fidx, sf, bidx, sb
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_all_stages(gpu_lib, name):
+    ci = SMALL[name]()
+    sh = ci.shape
+    t = G.to_dev(ci)
+    nbpf = O.n_blocks(sh.T, sh.block)
+
+    if sh.n_hist > 0:
+        qb, kb, kf, fidx, sf, bidx, sb = _oracle_selection(ci)
+        # (a) compression
+        g_qb, g_kb, g_kf = G.gpu_compress(ci, t)
+        for g, o in ((g_qb, qb), (g_kb, kb), (g_kf, kf)):
+            gn = g.cpu().double().numpy()
+            assert np.all(np.abs(gn - o) <= 2e-6 * (1 + np.abs(o))), name
+        # (b) frames, on the GPU's own pooled tensors
+        g_fidx, g_fsc = G.gpu_select_frames(ci, g_qb, g_kf)
+        assert np.allclose(g_fsc.cpu().double().numpy(), sf, rtol=1e-4, atol=1e-4)
+        kf_eff = min(sh.k_f, sh.n_hist)
+        bad, near, n = G.compare_indices(g_fidx.cpu().numpy(), fidx, G.frame_gaps(sf, kf_eff))
+        assert bad == 0, f"{name}: {bad}/{n} frame lists differ outside near ties"
+        # (c) blocks, isolated: the GPU selector on the oracle's frame lists
+        o_fidx = torch.as_tensor(fidx, dtype=torch.int32).cuda().contiguous()
+        g_bidx, g_bsc = G.gpu_select_blocks(ci, g_qb, g_kb, o_fidx)
+        assert np.allclose(g_bsc.cpu().double().numpy(), sb, rtol=1e-4, atol=1e-4)
+        kb_eff = min(sh.k_b, nbpf)
+        bad, near, n = G.compare_indices(g_bidx.cpu().numpy(), bidx, G.block_gaps(sb, kb_eff))
+        assert bad == 0, f"{name}: {bad}/{n} block lists differ outside near ties"
+        assert g_bidx.shape[-1] == kf_eff * kb_eff          # fixed complexity
+    else:
+        bidx = None
+
+    # (d) attention on the oracle's mask
+    o_ref, lse_ref = O.attention(sh, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                                 ci.hist_slots, ci.sink_slots, bidx)
+    out, lse = G.gpu_attention(ci, t, bidx)
+    torch.cuda.synchronize()
+    G.assert_output_close(out, o_ref, what=name)
+    assert np.abs(lse.cpu().double().numpy() - lse_ref).max() <= G.LSE_ABS
+
+    # end to end through lf_forward_chunk
+    out2, lse2, g_b2 = G.gpu_forward(ci, t)
+    torch.cuda.synchronize()
+    if sh.n_hist > 0:
+        g_b2 = g_b2.cpu().numpy()
+        same = np.all(g_b2 == bidx, axis=-1)                   # [H, nqb]
+        o_n = out2.float().cpu().double().numpy()
+        for h in range(sh.H):
+            for q in range(same.shape[1]):
+                if same[h, q]:
+                    rows = G.qblock_rows(sh.T, sh.block, q)
+                    err = np.abs(o_n[rows, h] - o_ref[rows, h]).max()
+                    assert err <= G.OUT_MAX_ABS, (name, h, q, err)
+        assert same.mean() >= 0.9, f"{name}: selections differ on {1 - same.mean():.2%}"
+    else:
+        G.assert_output_close(out2, o_ref, what=name + "/forward")
+    assert gpu_lib.lf_device_status() == 0
+
+
+def _full_size_check(ci, samples):
+    """The benchmark's call on a full-size workload; all indices against the oracle,
+    output on sampled query blocks (oracle attention given the GPU's own mask)."""
+    sh = ci.shape
+    t = G.to_dev(ci)
+    out, lse, g_bidx = G.gpu_forward(ci, t)
+    torch.cuda.synchronize()
+    o_n = out.float()
+    assert torch.isfinite(o_n).all() and torch.isfinite(lse).all()
+    g_bidx = g_bidx.cpu().numpy()
+    nbpf = O.n_blocks(sh.T, sh.block)
+    if sh.n_hist > 0:
+        qb, kb, kf, fidx, sf, bidx, sb = _oracle_selection(ci)
+        kf_eff, kb_eff = min(sh.k_f, sh.n_hist), min(sh.k_b, nbpf)
+        gaps = np.minimum(G.frame_gaps(sf, kf_eff), G.block_gaps(sb, kb_eff))
+        bad, near, n = G.compare_indices(g_bidx, bidx, gaps)
+        assert bad == 0, f"{ci.name}: {bad}/{n} block lists differ outside near ties ({near} near)"
+    rng = np.random.default_rng(0)
+    nqb = sh.n_cur_frames * nbpf
+    picks = {(0, 0), (sh.H - 1, nqb - 1), (sh.H // 2, nbpf - 1)}
+    while len(picks) < samples:
+        picks.add((int(rng.integers(sh.H)), int(rng.integers(nqb))))
+    for h, q in sorted(picks):
+        o_ref, lse_ref = O.attention(sh, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                                     ci.hist_slots, ci.sink_slots,
+                                     g_bidx if sh.n_hist > 0 else None, heads=[h], qblocks=[q])
+        rows = G.qblock_rows(sh.T, sh.block, q)
+        g = out[rows, h].float().cpu().double().numpy()
+        r = o_ref[rows, h]
+        err = g - r
+        assert np.abs(err).max() <= G.OUT_MAX_ABS, (ci.name, h, q)
+        assert np.linalg.norm(err) / np.linalg.norm(r) <= G.OUT_REL_L2, (ci.name, h, q)
+        assert np.abs(lse[h, rows].cpu().double().numpy() - lse_ref[h, rows]).max() <= G.LSE_ABS
+    return out
+
+
+def test_480p_chunk_full_size(gpu_lib):
+    ci = W.p480(0)
+    out = _full_size_check(ci, samples=16)
+    # determinism: the same call again gives the same bits
+    t = G.to_dev(ci)
+    out2, _, _ = G.gpu_forward(ci, t)
+    assert torch.equal(out, out2)
+    assert gpu_lib.lf_device_status() == 0
+
+
+@pytest.mark.slow
+def test_large_model_full_size(gpu_lib):
+    _full_size_check(W.large(0), samples=8)
+    assert gpu_lib.lf_device_status() == 0
+
+
+def test_rolling_steady_state_chunk(gpu_lib):
+    chunks = W.rolling(0, n_chunks=9)
+    for ci in chunks:
+        pass                           # chunk 9: 3 sinks + 21 rolling history frames
+    assert ci.shape.n_sink == 3 and ci.shape.n_hist == 21
+    _full_size_check(ci, samples=6)
+    assert gpu_lib.lf_device_status() == 0
+
+
+def test_growth_sweep_chunk(gpu_lib):
+    ci = W.growth_sweep(0)[2]          # chunk 3: 6 history frames, (k_f, k_b) = (6, 6)
+    _full_size_check(ci, samples=6)
+
+
+def test_bad_block_index_is_reported_and_dropped(gpu_lib):
+    ci = W.tiny(0)
+    t = G.to_dev(ci)
+    sh = ci.shape
+    qb, kb, kf, fidx, sf, bidx, sb = _oracle_selection(ci)
+    bad = bidx.copy()
+    bad[0, 0, 0] = sh.n_hist * 4 + 3          # out of range
+    gpu_lib.lf_device_status(True)
+    out, _ = G.gpu_attention(ci, t, bad)
+    torch.cuda.synchronize()
+    assert gpu_lib.lf_device_status(True) == 6          # LF_ERR_BAD_INDEX
+    assert torch.isfinite(out.float()).all()
