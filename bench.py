@@ -214,16 +214,39 @@ def run_lf(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
-    def step(record=False):
-        if record:
-            ev[0].record(stream)
+    def sel_stage():
         lf.lf_compress(sh, t["q"], t["k_cache"], ci.hist_slots, q_blk, k_blk, k_frm)
         lf.lf_select_frames(sh, q_blk, k_frm, fidx)
         lf.lf_select_blocks(sh, q_blk, k_blk, fidx, bidx)
-        if record:
-            ev[1].record(stream)
+
+    def att_stage():
         lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
                                 ci.hist_slots, ci.sink_slots, bidx, out, lse, ws)
+
+    # warm up eagerly, then capture each stage in a CUDA graph (removes host overhead
+    # between launches; the graphs replay exactly the kernels of the C-ABI calls)
+    for _ in range(3):
+        sel_stage()
+        att_stage()
+    torch.cuda.synchronize()
+    g_sel, g_att = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g_sel, stream=cap):
+            sel_stage()
+        with torch.cuda.graph(g_att, stream=cap):
+            att_stage()
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+
+    def step(record=False):
+        if record:
+            ev[0].record(stream)
+        g_sel.replay()
+        if record:
+            ev[1].record(stream)
+        g_att.replay()
         if record:
             ev[2].record(stream)
 
@@ -280,11 +303,18 @@ def run_lf(args, rank, world, local_rank):
     for _ in range(3):
         e2e_step()
     torch.cuda.synchronize()
+    g_e2e = torch.cuda.CUDAGraph()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g_e2e, stream=cap):
+            e2e_step()
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0.record(stream)
     for _ in range(n_e2e):
-        e2e_step()
+        g_e2e.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
@@ -320,7 +350,7 @@ def run_lf(args, rank, world, local_rank):
                                "peak_source": f"{src} hbm_gbs"},
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "lf_forward_chunk"},
+                "api": "lf_forward_chunk (replayed as one CUDA graph with the copies)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }

@@ -147,6 +147,10 @@ int launch_attn_t(const Dims& D, lf::AttnParams& p, cudaStream_t st) {
   auto kern = lf::attn_kernel<HD, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return LF_ERR_CUDA;
+  // the in-kernel register split assumes the launch register count; never launch otherwise
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return LF_ERR_CUDA;
+  if (fa.numRegs != lf::kLaunchRegs) return LF_ERR_UNSUPPORTED;
   dim3 grid(lf::tile_count(D), D.H);
   kern<<<grid, lf::kAttnThreads, L::kAlloc, st>>>(p, D);
   return cuda_status(cudaGetLastError());
@@ -343,6 +347,13 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
   return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, bidx, out,
                      lse, w.attn, stream);
 }
+
+#ifdef LF_TRACE
+int lf_debug_set_trace(void* buf) {
+  unsigned long long* p = static_cast<unsigned long long*>(buf);
+  return cudaMemcpyToSymbol(lf::g_lf_trace, &p, sizeof(p)) == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}
+#endif
 
 int lf_device_status(int reset) {
   int v = 0;

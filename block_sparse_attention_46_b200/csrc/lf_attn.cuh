@@ -30,7 +30,7 @@
 namespace lf {
 
 constexpr int kMaxPlan = 2048;          // key-plan entries per query tile
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 384;
 
 // Plan entry: bits 0-1 = which of the tile's two query blocks selected it (bit 0: rows
 // 0-63 or the single 128-row block; bit 1: rows 64-127), bits 4-15 = block in frame,
@@ -150,22 +150,29 @@ struct AttnLayout {
   static constexpr int kK = kQ + kQBytes;            // K stages
   static constexpr int kStageBytes = NH * kRegion;
   static constexpr int kV = kK + 2 * kStageBytes;    // V stages
-  static constexpr int kP = kV + 2 * kStageBytes;    // P: 2 key halves x 128 rows x 128 B
-  static constexpr int kPBytes = 2 * kRegion;
-  static constexpr int kPlan = kP + kPBytes;
-  static constexpr int kBar = kPlan + kMaxPlan * 4;
+  static constexpr int kPlan = kV + 2 * kStageBytes;
+  static constexpr int kRed = kPlan + kMaxPlan * 4;  // per-row (m, l) of both warpgroups
+  static constexpr int kBar = kRed + 2 * 2 * 128 * 4;
   static constexpr int kNumBars = 16;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;       // slack for 1024-byte alignment
-  // tensor-memory columns
-  static constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kTmemCols = 512;
+  // tensor-memory columns: two O accumulators (one per softmax warpgroup), two S buffers;
+  // P (bf16 pairs) overwrites the first 64 columns of the S buffer it was computed from
+  static constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS0 = 256, kColS1 = 384,
+                            kTmemCols = 512;
 };
 
 enum BarId {
   kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7,
-  kBarSFull = 9, kBarSEmpty = 11, kBarPFull = 13, kBarODone = 14, kBarDrain = 15
+  kBarSFull = 9, kBarPFull = 11, kBarDone = 13
 };
+
+constexpr int kSoftmaxWarps = 8;          // two warpgroups, alternate key tiles
+// Register split: launched at 168 per thread (384 threads); the load/MMA warpgroup gives
+// registers to the two softmax warpgroups: 128 x 72 + 256 x 216 <= 384 x 168.
+constexpr int kLaunchRegs = 168, kLowRegs = 72, kHighRegs = 216;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kAttnThreads * kLaunchRegs, "register split");
 
 template <int HD, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -176,6 +183,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint32_t* s_plan = reinterpret_cast<uint32_t*>(smem + L::kPlan);
+  float* s_red = reinterpret_cast<float*>(smem + L::kRed);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -202,11 +210,9 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       mbar_init(&bars[kBarVFull + s], 1);
       mbar_init(&bars[kBarVEmpty + s], 1);
       mbar_init(&bars[kBarSFull + s], 1);
-      mbar_init(&bars[kBarSEmpty + s], 4);
+      mbar_init(&bars[kBarPFull + s], 4);
     }
-    mbar_init(&bars[kBarPFull], 4);
-    mbar_init(&bars[kBarODone], 1);
-    mbar_init(&bars[kBarDrain], 1);
+    mbar_init(&bars[kBarDone], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -229,6 +235,8 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
+  if (warp < 4) {
+  regs_dec<kLowRegs>();
   // -------------------------------------------------------------- producers
   if ((warp == 0 || warp == 2) && lane == 0) {
     const bool isK = warp == 0;
@@ -250,6 +258,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     for (; j < n_iter; ++j) {
       const int s = j & 1;
       if (j >= 2 && !mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, s_abort)) break;
+      LF_TR(isK ? 0 : 1, j);
       mbar_arrive_expect_tx(&full[s], L::kStageBytes);
       uint8_t* st = stage0 + s * L::kStageBytes;
       for (int box = 0; box < 2; ++box) {
@@ -280,81 +289,85 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     }
   }
   // -------------------------------------------------------------- MMA issuer
+  // Order: S0, S1, then for each i: PV_i (O_{i&1} += P_i V_i), S_{i+2} into the S buffer
+  // P_i was read from.  tcgen05.mma runs in issue order, so S_{i+2} overwrites P_i only
+  // after PV_i has consumed it, and the completion of S_{i+2} implies that of PV_i.
   else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, 0, 1);
     const uint32_t q_base = smem_u32(smem + L::kQ);
     const uint32_t k_base = smem_u32(smem + L::kK);
     const uint32_t v_base = smem_u32(smem + L::kV);
-    const uint32_t p_base = smem_u32(smem + L::kP);
+    auto issue_s = [&](int j) -> bool {
+      const int s = j & 1;
+      LF_TR(2, j);
+      if (!mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, s_abort)) return false;
+      LF_TR(3, j);
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
+        mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
+                    smem_desc_sw128(k_base + s * L::kStageBytes + off, 16, 1024),
+                    idesc_qk, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(&bars[kBarSFull + s]);
+      mma_commit(&bars[kBarKEmpty + s]);
+      return true;
+    };
     bool ok = mbar_wait(&bars[kBarQ], 0, s_abort);
-    for (int j = 0; ok && j <= n_iter; ++j) {
-      if (j < n_iter) {
-        const int s = j & 1;
-        ok = mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, s_abort);
-        if (ok && j >= 2) ok = mbar_wait(&bars[kBarSEmpty + s], ((j >> 1) & 1) ^ 1, s_abort);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
+    if (ok) ok = issue_s(0);
+    if (ok && n_iter > 1) ok = issue_s(1);
+    for (int i = 0; ok && i < n_iter; ++i) {
+      const int s = i & 1;
+      ok = mbar_wait(&bars[kBarVFull + s], (i >> 1) & 1, s_abort);
+      LF_TR(4, i);
+      if (ok) ok = mbar_wait(&bars[kBarPFull + s], (i >> 1) & 1, s_abort);
+      if (!ok) break;
+      LF_TR(5, i);
+      tc_fence_after();
+      const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
+      const uint32_t o_tmem = tmem + (s ? L::kColO1 : L::kColO0);
 #pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
-          mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
-                      smem_desc_sw128(k_base + s * L::kStageBytes + off, 16, 1024),
-                      idesc_qk, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[kBarSFull + s]);
-        mma_commit(&bars[kBarKEmpty + s]);
-      }
-      if (j >= 1) {
-        const int i = j - 1, s = i & 1;
-        ok = mbar_wait(&bars[kBarVFull + s], (i >> 1) & 1, s_abort);
-        if (ok) ok = mbar_wait(&bars[kBarPFull], i & 1, s_abort);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {          // 128 keys, 16 per MMA
-          const uint32_t a_off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
-          const uint32_t b_off = ks * 16 * 128;
-          mma_bf16_ss(tmem + L::kColO, smem_desc_sw128(p_base + a_off, 16, 1024),
-                      smem_desc_sw128(v_base + s * L::kStageBytes + b_off, L::kRegion, 1024),
-                      idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars[kBarODone]);
-        mma_commit(&bars[kBarVEmpty + s]);
-      }
+      for (int ks = 0; ks < 8; ++ks)            // 128 keys, 16 per MMA, 8 columns each
+        mma_bf16_ts(o_tmem, p_tmem + ks * 8,
+                    smem_desc_sw128(v_base + s * L::kStageBytes + ks * 16 * 128, L::kRegion, 1024),
+                    idesc_pv, (i >= 2 || ks > 0) ? 1u : 0u);
+      mma_commit(&bars[kBarVEmpty + s]);
+      if (i + 2 < n_iter) ok = issue_s(i + 2);
     }
-    // drain: all MMAs issued by this thread complete before tensor memory is released
-    mma_commit(&bars[kBarDrain]);
-    mbar_wait_drain(&bars[kBarDrain], 0);
+    // completion of everything issued: epilogue may read O, tensor memory may be freed
+    mma_commit(&bars[kBarDone]);
   }
+  } else {
+  regs_inc<kHighRegs>();
   // -------------------------------------------------------------- softmax + epilogue
-  else if (warp >= 4) {
-    const int r = threadIdx.x - 128;                       // query row = TMEM lane
+  {
+    const int wg = (warp - 4) >> 2;                        // handles key tiles j = wg, wg+2, ...
+    const int r = (threadIdx.x - 128) & 127;               // query row = TMEM lane
     const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t row_bit = (BLK == 64 && r >= 64) ? 2u : 1u;
+    const uint32_t s_col = wg ? L::kColS1 : L::kColS0;
+    const uint32_t o_col = wg ? L::kColO1 : L::kColO0;
     const float c = D.scale * 1.4426950408889634f;         // scale * log2(e)
-    uint8_t* p_smem = smem + L::kP;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int j = 0;
-    for (; j < n_iter; ++j) {
-      const int s = j & 1;
-      ok = mbar_wait(&bars[kBarSFull + s], (j >> 1) & 1, s_abort);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+    int n_mine = 0;                                        // PVs into this group's O
+    for (int j = wg; j < n_iter; j += 2, ++n_mine) {
+      if (threadIdx.x == 128) LF_TR(6, j);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + wg], (j >> 1) & 1, s_abort)) && ok;
+      if (threadIdx.x == 128) LF_TR(7, j);
       tc_fence_after();
       float sv[128];
-      const uint32_t s_col = s ? L::kColS1 : L::kColS0;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) tmem_ld32(t_row + s_col + ch * 32, sv + ch * 32);
       tmem_ld_wait();
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) reg_fence32(sv + ch * 32);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarSEmpty + s]);
+      if (threadIdx.x == 128) LF_TR(8, j);
 
-      // valid key columns of this row: [0, v0) in the first 64, [64, 64 + v1) in the second
+      // valid key columns of this row: [0, v0) and [64, 64 + v1)
       int v0, v1;
       if (j < n_dense) {
         const int n = min(128, D.ncur - j * 128);
@@ -379,109 +392,123 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
           v1 = max(0, len - 64);
         }
       }
-      float mx = -INFINITY;
+      if (v0 < 64 || v1 < 64) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        if (i >= v0) sv[i] = -INFINITY;
-        if (i >= v1) sv[64 + i] = -INFINITY;
+        for (int i = 0; i < 64; ++i) {
+          if (i >= v0) sv[i] = -INFINITY;
+          if (i >= v1) sv[64 + i] = -INFINITY;
+        }
       }
+      float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) mx = fmaxf(mx, sv[i]);
-      const float m_tile = mx * c;
+      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(sv[k], sv[8 + k]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], sv[i + k]);
+      const float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * c;
       float m_new = m_run;
       bool resc = false;
       if (m_tile > m_run + 8.0f) { m_new = m_tile; resc = true; }
-      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
-
-      // PV of the previous tile must be done: P buffer reuse and O rescale
-      if (j > 0) {
-        ok = mbar_wait(&bars[kBarODone], (j - 1) & 1, s_abort);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          const float a = resc ? alpha : 1.f;
+      // lazy rescale of this group's O: its previous PV (PV_{j-2}) completed before S_j did
+      if (n_mine > 0 && __any_sync(0xffffffffu, resc)) {
+        const float a = resc ? exp2f(m_run - m_new) : 1.f;
 #pragma unroll
-          for (int ch = 0; ch < HD / 32; ++ch) {
-            float o[32];
-            tmem_ld32(t_row + L::kColO + ch * 32, o);
-            tmem_ld_wait();
-            reg_fence32(o);
+        for (int ch = 0; ch < HD / 32; ++ch) {
+          float o[32];
+          tmem_ld32(t_row + o_col + ch * 32, o);
+          tmem_ld_wait();
+          reg_fence32(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= a;
-            tmem_st32(t_row + L::kColO + ch * 32, o);
-          }
-          tmem_st_wait();
+          for (int q = 0; q < 32; ++q) o[q] *= a;
+          tmem_st32(t_row + o_col + ch * 32, o);
         }
+        if (resc) l_run *= a;
       }
-      if (resc) l_run *= alpha;
+      if (threadIdx.x == 128) LF_TR(9, j);
       const float mref = (m_new == -INFINITY) ? 0.f : m_new;
-      float psum = 0.f;
-      uint8_t* prow = p_smem + r * 128;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int kh = 0; kh < 2; ++kh) {
+      for (int half = 0; half < 2; ++half) {
+        float pk[32];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2_approx(fmaf(sv[kh * 64 + cc * 8 + 2 * e], c, -mref));
-            const float p1 = ex2_approx(fmaf(sv[kh * 64 + cc * 8 + 2 * e + 1], c, -mref));
-            psum += p0 + p1;
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            pk[e] = *reinterpret_cast<uint32_t*>(&b2);
-          }
-          const int chunk = cc ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + kh * L::kRegion + chunk * 16) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = ex2_approx(fmaf(sv[half * 64 + 2 * e], c, -mref));
+          const float p1 = ex2_approx(fmaf(sv[half * 64 + 2 * e + 1], c, -mref));
+          ps[e & 3] += p0 + p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&b2));
         }
+        tmem_st32(t_row + s_col + half * 32, pk);
       }
-      l_run += psum;
+      if (threadIdx.x == 128) LF_TR(10, j);
+      tmem_st_wait();
+      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       m_run = m_new;
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarPFull]);
+      if (lane == 0) mbar_arrive(&bars[kBarPFull + wg]);
+      if (threadIdx.x == 128) LF_TR(11, j);
     }
-    if (ok && n_iter > 0) {
-      ok = mbar_wait(&bars[kBarODone], (n_iter - 1) & 1, s_abort);
-      ok = __all_sync(0xffffffffu, ok);
-    }
+    ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0, s_abort)) && ok;
+    // merge the two groups' partial softmax states: O = sum_w 2^(m_w - m) O_w / l
+    s_red[wg * 128 + r] = m_run;
+    s_red[256 + wg * 128 + r] = l_run;
+    named_bar_sync(1, kSoftmaxWarps * 32);
+    const float m_o = s_red[(wg ^ 1) * 128 + r], l_o = s_red[256 + (wg ^ 1) * 128 + r];
+    const float m_all = fmaxf(m_run, m_o);
+    const float w_me = m_run == -INFINITY ? 0.f : exp2f(m_run - m_all);
+    const float w_o = m_o == -INFINITY ? 0.f : exp2f(m_o - m_all);
+    const float l_tot = l_run * w_me + l_o * w_o;
     if (ok) {
       tc_fence_after();
-      // output row
       int qb, i;
       if (BLK == 64) { qb = r < 64 ? qbA : qbB; i = r & 63; }
       else { qb = qbA; i = r; }
       const bool valid = qb >= 0 && i < block_len(D, qb % D.nbpf);
       const int tok = qb >= 0 ? (qb / D.nbpf) * D.T + (qb % D.nbpf) * BLK + i : 0;
-      const float inv_l = 1.0f / l_run;
-      __nv_bfloat16* orow = P.out + ((size_t)tok * D.H + h) * HD;
+      const float inv_l = 1.0f / l_tot;
+      // this group writes output columns [wg*HD/2, (wg+1)*HD/2) from both accumulators
+      const float w0 = (wg == 0 ? w_me : w_o) * inv_l, w1 = (wg == 0 ? w_o : w_me) * inv_l;
+      __nv_bfloat16* orow = P.out + ((size_t)tok * D.H + h) * HD + wg * (HD / 2);
 #pragma unroll
-      for (int ch = 0; ch < HD / 32; ++ch) {
-        float o[32];
-        tmem_ld32(t_row + L::kColO + ch * 32, o);
+      for (int ch = 0; ch < HD / 64; ++ch) {
+        float a[32], b[32];
+        const uint32_t col = wg * (HD / 2) + ch * 32;
+        tmem_ld32(t_row + L::kColO0 + col, a);
+        tmem_ld32(t_row + L::kColO1 + col, b);
         tmem_ld_wait();
-        reg_fence32(o);
+        reg_fence32(a);
+        reg_fence32(b);
         if (valid) {
-          uint32_t pk[16];
+          uint32_t pw[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
-            pk[e] = *reinterpret_cast<uint32_t*>(&b2);
+            // a group that never accumulated has weight 0 and its O is not read into the sum
+            const float x0 = (w0 > 0.f ? a[2 * e] * w0 : 0.f) + (w1 > 0.f ? b[2 * e] * w1 : 0.f);
+            const float x1 = (w0 > 0.f ? a[2 * e + 1] * w0 : 0.f) +
+                             (w1 > 0.f ? b[2 * e + 1] * w1 : 0.f);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+            pw[e] = *reinterpret_cast<uint32_t*>(&b2);
           }
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            dst[e] = make_uint4(pw[4 * e], pw[4 * e + 1], pw[4 * e + 2], pw[4 * e + 3]);
         }
       }
-      if (valid && P.lse != nullptr)
-        P.lse[(size_t)h * D.ncur + tok] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+      if (valid && wg == 0 && P.lse != nullptr)
+        P.lse[(size_t)h * D.ncur + tok] = (m_all + log2f(l_tot)) * 0.6931471805599453f;
       tc_fence_before();
     }
   }
+  }
   __syncthreads();
   if (warp == 1) {
+    // everything the MMA thread issued is complete before tensor memory is released
+    if (lane == 0) mbar_wait_drain(&bars[kBarDone], 0);
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }

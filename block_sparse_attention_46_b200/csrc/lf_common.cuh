@@ -38,6 +38,22 @@ __device__ __forceinline__ void record_status(int code) {
   atomicCAS(&g_lf_status, 0, code);
 }
 
+// Optional pipeline trace (compiled in only with -DLF_TRACE): SM clock stamps of named
+// events of the first traced CTAs, written to a caller-registered buffer.
+#ifdef LF_TRACE
+__device__ unsigned long long* g_lf_trace = nullptr;
+constexpr int kTraceCtas = 4, kTraceEvents = 16, kTraceIters = 256;
+#define LF_TR(ev, it)                                                                    \
+  do {                                                                                   \
+    const int _cta = blockIdx.x + blockIdx.y * gridDim.x;                                \
+    if (g_lf_trace && _cta < lf::kTraceCtas && (it) < lf::kTraceIters)                   \
+      g_lf_trace[((size_t)_cta * lf::kTraceEvents + (ev)) * lf::kTraceIters + (it)] =    \
+          clock64();                                                                     \
+  } while (0)
+#else
+#define LF_TR(ev, it) do {} while (0)
+#endif
+
 // ------------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -83,6 +99,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (*abort) return false;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -174,6 +191,32 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// D(tmem) (+)= A(tmem) * B(smem desc)^T, kind::f16: A is M x K bf16 in tensor memory,
+// two consecutive K elements per 32-bit column (row m in lane m).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Per-warp register budget changes (whole warpgroups; the sum over the CTA must stay
+// within the launch's registers: threads x registers per thread at launch).
+template <uint32_t N> __device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N> __device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Named barrier over `nthreads` threads (id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Arrive (once) on an mbarrier when every tcgen05 op issued so far by this thread is done.
