@@ -147,13 +147,14 @@ struct AttnLayout {
   static constexpr int kRegion = 128 * 128;          // bytes of one 128-row x 64-col half
   static constexpr int kQ = 0;
   static constexpr int kQBytes = NH * kRegion;
-  static constexpr int kK = kQ + kQBytes;            // K stages
+  // one ring of K and V tiles in the order the MMAs consume them: K0, K1, V0, K2, V1, ...
+  static constexpr int kSlots = HD == 128 ? 5 : 10;
+  static constexpr int kRing = kQ + kQBytes;
   static constexpr int kStageBytes = NH * kRegion;
-  static constexpr int kV = kK + 2 * kStageBytes;    // V stages
-  static constexpr int kPlan = kV + 2 * kStageBytes;
+  static constexpr int kPlan = kRing + kSlots * kStageBytes;
   static constexpr int kRed = kPlan + kMaxPlan * 4;  // per-row (m, l) of both warpgroups
   static constexpr int kBar = kRed + 2 * 2 * 128 * 4;
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 2 * kSlots + 8;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;       // slack for 1024-byte alignment
@@ -163,10 +164,19 @@ struct AttnLayout {
                             kTmemCols = 512;
 };
 
-enum BarId {
-  kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7,
-  kBarSFull = 9, kBarPFull = 11, kBarDone = 13
-};
+// barrier indices: ring full/empty barriers follow these
+enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 5, kBarRing = 6 };
+
+// position of a tile in the ring's load order: K0, K1, V0, K2, V1, K3, V2, ...
+__device__ __forceinline__ int ring_pos_k(int j) { return j < 2 ? j : 2 * j - 1; }
+__device__ __forceinline__ int ring_pos_v(int i) { return 2 + 2 * i; }
+// inverse: the tile at ring position q (K_j when isK, else V_j)
+__device__ __forceinline__ int ring_tile(int q, bool& isK) {
+  if (q < 2) { isK = true; return q; }
+  if ((q & 1) == 0) { isK = false; return (q - 2) >> 1; }
+  isK = true;
+  return (q + 1) >> 1;
+}
 
 constexpr int kSoftmaxWarps = 8;          // two warpgroups, alternate key tiles
 // Register split: launched at 168 per thread (384 threads); the load/MMA warpgroup gives
@@ -205,13 +215,10 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarQ], 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[kBarKFull + s], 1);
-      mbar_init(&bars[kBarKEmpty + s], 1);
-      mbar_init(&bars[kBarVFull + s], 1);
-      mbar_init(&bars[kBarVEmpty + s], 1);
       mbar_init(&bars[kBarSFull + s], 1);
       mbar_init(&bars[kBarPFull + s], 4);
     }
+    for (int q = 0; q < 2 * L::kSlots; ++q) mbar_init(&bars[kBarRing + q], 1);
     mbar_init(&bars[kBarDone], 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -226,8 +233,6 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&P.tm_q); prefetch_tmap(&P.tm_kc); prefetch_tmap(&P.tm_kh);
-  }
-  if (warp == 2 && lane == 0) {
     prefetch_tmap(&P.tm_vc); prefetch_tmap(&P.tm_vh);
   }
   tc_fence_before();
@@ -237,55 +242,58 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
 
   if (warp < 4) {
   regs_dec<kLowRegs>();
-  // -------------------------------------------------------------- producers
-  if ((warp == 0 || warp == 2) && lane == 0) {
-    const bool isK = warp == 0;
-    const CUtensorMap* tm_cur = isK ? &P.tm_kc : &P.tm_vc;
-    const CUtensorMap* tm_hist = isK ? &P.tm_kh : &P.tm_vh;
-    uint64_t* full = &bars[isK ? kBarKFull : kBarVFull];
-    uint64_t* empty = &bars[isK ? kBarKEmpty : kBarVEmpty];
-    uint8_t* stage0 = smem + (isK ? L::kK : L::kV);
-    if (isK) {
-      mbar_arrive_expect_tx(&bars[kBarQ], L::kQBytes);
-      for (int c = 0; c < L::NH; ++c) {
-        uint8_t* dst = smem + L::kQ + c * L::kRegion;
-        tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD + c * 64, tokA);
-        tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD + c * 64,
-                    BLK == 64 ? tokB : tokA + 64);
-      }
+  // -------------------------------------------------------------- producer
+  if (warp == 0 && lane == 0) {
+    uint64_t* full = &bars[kBarRing];
+    uint64_t* empty = &bars[kBarRing + L::kSlots];
+    mbar_arrive_expect_tx(&bars[kBarQ], L::kQBytes);
+    for (int c = 0; c < L::NH; ++c) {
+      uint8_t* dst = smem + L::kQ + c * L::kRegion;
+      tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD + c * 64, tokA);
+      tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD + c * 64,
+                  BLK == 64 ? tokB : tokA + 64);
     }
-    int j = 0;
-    for (; j < n_iter; ++j) {
-      const int s = j & 1;
-      if (j >= 2 && !mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, s_abort)) break;
+    const int n_pos = 2 * n_iter + 1;               // V_{n-1} sits at position 2n
+    int q = 0;
+    for (; q < n_pos; ++q) {
+      bool isK;
+      const int j = ring_tile(q, isK);
+      const int slot = q % L::kSlots;
+      const int rnd = q / L::kSlots;
+      if (isK && j >= n_iter) continue;            // no slot used, nothing to load
+      if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort)) break;
       LF_TR(isK ? 0 : 1, j);
-      mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-      uint8_t* st = stage0 + s * L::kStageBytes;
+      mbar_arrive_expect_tx(&full[slot], L::kStageBytes);
+      uint8_t* st = smem + L::kRing + slot * L::kStageBytes;
+      const CUtensorMap* tm_cur = isK ? &P.tm_kc : &P.tm_vc;
+      const CUtensorMap* tm_hist = isK ? &P.tm_kh : &P.tm_vh;
       for (int box = 0; box < 2; ++box) {
         if (j < n_dense) {
           const int row = j * 128 + box * 64;
           for (int c = 0; c < L::NH; ++c)
-            tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[s],
+            tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
                         h * HD + c * 64, row);
         } else {
           const int u = j - n_dense;
-          int slot = 0, tok = D.T;                      // default: all rows out of bounds
+          int slot_id = 0, tok = D.T;                   // default: all rows out of bounds
           const int e = BLK == 64 ? 2 * u + box : u;
           if (e < cnt) {
             const uint32_t pe = s_plan[e];
-            slot = P.slots[pe >> 16];
+            slot_id = P.slots[pe >> 16];
             tok = (int)((pe >> 4) & 0xFFFu) * BLK + (BLK == 64 ? 0 : box * 64);
           }
           for (int c = 0; c < L::NH; ++c)
-            tma_load_3d(st + c * L::kRegion + box * 64 * 128, tm_hist, &full[s],
-                        h * HD + c * 64, tok, slot);
+            tma_load_3d(st + c * L::kRegion + box * 64 * 128, tm_hist, &full[slot],
+                        h * HD + c * 64, tok, slot_id);
         }
       }
     }
-    // drain: every load issued must land before the CTA may exit
-    for (int s = 0; s < 2; ++s) {
-      const int last = (j - 1 - s) >= 0 ? ((j - 1 - s) & ~1) + s : -1;
-      if (last >= 0) mbar_wait_drain(&full[s], (last >> 1) & 1);
+    // drain: every load issued must land before the CTA may exit (the last kSlots
+    // positions hold the only loads that nobody may have waited for)
+    for (int x = max(0, q - L::kSlots); x < q; ++x) {
+      bool isK;
+      const int jx = ring_tile(x, isK);
+      if (!(isK && jx >= n_iter)) mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1);
     }
   }
   // -------------------------------------------------------------- MMA issuer
@@ -296,24 +304,26 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, 0, 1);
     const uint32_t q_base = smem_u32(smem + L::kQ);
-    const uint32_t k_base = smem_u32(smem + L::kK);
-    const uint32_t v_base = smem_u32(smem + L::kV);
+    const uint32_t ring_base = smem_u32(smem + L::kRing);
+    uint64_t* full = &bars[kBarRing];
+    uint64_t* empty = &bars[kBarRing + L::kSlots];
     auto issue_s = [&](int j) -> bool {
       const int s = j & 1;
+      const int q = ring_pos_k(j), slot = q % L::kSlots;
       LF_TR(2, j);
-      if (!mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, s_abort)) return false;
+      if (!mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort)) return false;
       LF_TR(3, j);
       tc_fence_after();
       const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
+      const uint32_t k_addr = ring_base + slot * L::kStageBytes;
 #pragma unroll
       for (int ks = 0; ks < HD / 16; ++ks) {
         const uint32_t off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
         mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
-                    smem_desc_sw128(k_base + s * L::kStageBytes + off, 16, 1024),
-                    idesc_qk, ks > 0 ? 1u : 0u);
+                    smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
       }
       mma_commit(&bars[kBarSFull + s]);
-      mma_commit(&bars[kBarKEmpty + s]);
+      mma_commit(&empty[slot]);
       return true;
     };
     bool ok = mbar_wait(&bars[kBarQ], 0, s_abort);
@@ -321,7 +331,8 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     if (ok && n_iter > 1) ok = issue_s(1);
     for (int i = 0; ok && i < n_iter; ++i) {
       const int s = i & 1;
-      ok = mbar_wait(&bars[kBarVFull + s], (i >> 1) & 1, s_abort);
+      const int qv = ring_pos_v(i), vslot = qv % L::kSlots;
+      ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort);
       LF_TR(4, i);
       if (ok) ok = mbar_wait(&bars[kBarPFull + s], (i >> 1) & 1, s_abort);
       if (!ok) break;
@@ -332,9 +343,10 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)            // 128 keys, 16 per MMA, 8 columns each
         mma_bf16_ts(o_tmem, p_tmem + ks * 8,
-                    smem_desc_sw128(v_base + s * L::kStageBytes + ks * 16 * 128, L::kRegion, 1024),
+                    smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
+                                    L::kRegion, 1024),
                     idesc_pv, (i >= 2 || ks > 0) ? 1u : 0u);
-      mma_commit(&bars[kBarVEmpty + s]);
+      mma_commit(&empty[vslot]);
       if (i + 2 < n_iter) ok = issue_s(i + 2);
     }
     // completion of everything issued: epilogue may read O, tensor memory may be freed
@@ -401,13 +413,15 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       }
       float mx8[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(sv[k], sv[8 + k]);
+      for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(sv[k], sv[8 + k], sv[16 + k]);
 #pragma unroll
-      for (int i = 16; i < 128; i += 8)
+      for (int i = 24; i < 120; i += 16)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], sv[i + k]);
-      const float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * c;
+        for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(mx8[k], sv[i + k], sv[i + 8 + k]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], sv[120 + k]);
+      const float m_tile = fmaxf(fmax3f(mx8[0], mx8[1], mx8[2]),
+                                 fmax3f(fmax3f(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * c;
       float m_new = m_run;
       bool resc = false;
       if (m_tile > m_run + 8.0f) { m_new = m_tile; resc = true; }

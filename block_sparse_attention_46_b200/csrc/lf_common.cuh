@@ -128,6 +128,13 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max.f32).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32; 2^-inf = 0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
