@@ -59,6 +59,7 @@ _SIGS = {
     "lf_device_status": (ctypes.c_int, [ctypes.c_int]),
     "lf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "lf_abi_version": (ctypes.c_int, []),
+    "lf_debug_exp2_poly": (ctypes.c_int, [_P, _P, ctypes.c_int, _P]),
 }
 
 
@@ -126,6 +127,12 @@ def lf_abi_version() -> int:
 
 def lf_device_status(reset: bool = True) -> int:
     return load().lf_device_status(1 if reset else 0)
+
+
+def lf_debug_exp2_poly(x, y, stream=None):
+    """Test hook: the attention softmax's FMA-pipe exponential, y = 2^x (x <= 0)."""
+    _check(load().lf_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "lf_debug_exp2_poly")
 
 
 def lf_compress(shape, q, k_cache, hist_slots, q_blk, k_blk, k_frm, stream=None):

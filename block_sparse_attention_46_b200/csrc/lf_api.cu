@@ -135,14 +135,70 @@ int launch_select_blocks(const Dims& D, const float* q_blk, const float* k_blk,
   return cuda_status(cudaGetLastError());
 }
 
-size_t attn_ws_bytes(const Dims& D) {
-  const size_t nt = (size_t)lf::tile_count(D) * D.H;
-  return align_up(nt * lf::plan_stride(D) * sizeof(uint32_t), 256) +
-         align_up(nt * sizeof(int32_t), 256);
+// SM count of the current device (work decomposition and workspace sizing).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
 }
 
+// Work decomposition of the attention grid: full waves of whole tiles; if the last wave
+// would be less than half full, its tiles are split into `pieces` key ranges each.
+struct Split {
+  int n_whole, n_tail, pieces;
+};
+
+Split make_split(const Dims& D, int n_sm) {
+  const int ntot = lf::tile_count(D) * D.H;
+  Split sp{ntot, 0, 1};
+  if (n_sm <= 0) return sp;
+  const int R = ntot % n_sm;
+#ifdef LF_NO_TAIL_SPLIT
+  return sp;
+#endif
+  if (R == 0 || 2 * R > n_sm) return sp;
+  int p = n_sm / R;
+  p = p < 16 ? p : 16;
+  const int n_dense = lf::cdiv(D.ncur, 128);      // every tile has at least this many
+  p = p < n_dense ? p : n_dense;
+  if (p < 2) return sp;
+  sp.n_whole = ntot - R;
+  sp.n_tail = R;
+  sp.pieces = p;
+  return sp;
+}
+
+struct AttnWs {
+  uint32_t* plan;
+  int32_t* plan_cnt;
+  int32_t* order;
+  float* part_o;
+  float* part_ml;
+  size_t bytes;
+};
+
+// plan | counts | partial O of up to n_sm pieces | their (m, l)
+AttnWs carve_attn(const Dims& D, void* base, int n_sm) {
+  AttnWs w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t n) { uint8_t* r = p ? p + off : nullptr; off += align_up(n, 256); return r; };
+  const size_t nt = (size_t)lf::tile_count(D) * D.H;
+  const size_t units = n_sm > 0 ? (size_t)n_sm : 0;
+  w.plan = reinterpret_cast<uint32_t*>(take(nt * lf::plan_stride(D) * sizeof(uint32_t)));
+  w.plan_cnt = reinterpret_cast<int32_t*>(take(nt * sizeof(int32_t)));
+  w.order = reinterpret_cast<int32_t*>(take(nt * sizeof(int32_t)));
+  w.part_o = reinterpret_cast<float*>(take(units * 128 * D.d * sizeof(float)));
+  w.part_ml = reinterpret_cast<float*>(take(units * 2 * 128 * sizeof(float)));
+  w.bytes = off;
+  return w;
+}
+
+size_t attn_ws_bytes(const Dims& D) { return carve_attn(D, nullptr, sm_count()).bytes; }
+
 template <int HD, int BLK>
-int launch_attn_t(const Dims& D, lf::AttnParams& p, cudaStream_t st) {
+int launch_attn_t(const Dims& D, lf::AttnParams& p, int grid, cudaStream_t st) {
   using L = lf::AttnLayout<HD>;
   auto kern = lf::attn_kernel<HD, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -151,7 +207,6 @@ int launch_attn_t(const Dims& D, lf::AttnParams& p, cudaStream_t st) {
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return LF_ERR_CUDA;
   if (fa.numRegs != lf::kLaunchRegs) return LF_ERR_UNSUPPORTED;
-  dim3 grid(lf::tile_count(D), D.H);
   kern<<<grid, lf::kAttnThreads, L::kAlloc, st>>>(p, D);
   return cuda_status(cudaGetLastError());
 }
@@ -160,12 +215,12 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
                 const void* k_cache, const void* v_cache, const int32_t* hist_slots,
                 const int32_t* sink_slots, const int32_t* block_idx, void* out, float* lse,
                 void* workspace, cudaStream_t st) {
-  const size_t nt = (size_t)lf::tile_count(D) * D.H;
-  uint32_t* plan = static_cast<uint32_t*>(workspace);
-  int32_t* plan_cnt = reinterpret_cast<int32_t*>(
-      static_cast<uint8_t*>(workspace) + align_up(nt * lf::plan_stride(D) * sizeof(uint32_t), 256));
+  const int n_sm = sm_count();
+  if (n_sm <= 0) return LF_ERR_CUDA;
+  const AttnWs w = carve_attn(D, workspace, n_sm);
   lf::plan_kernel<<<dim3(lf::tile_count(D), D.H), 32, 0, st>>>(
-      D.F > 0 ? block_idx : nullptr, plan, plan_cnt, D);
+      D.F > 0 ? block_idx : nullptr, w.plan, w.plan_cnt, D);
+  lf::schedule_kernel<<<1, 1024, 0, st>>>(w.plan_cnt, w.order, D);
   int rc = cuda_status(cudaGetLastError());
   if (rc != LF_OK) return rc;
 
@@ -182,14 +237,27 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
     p.tm_kh = p.tm_kc;
     p.tm_vh = p.tm_vc;
   }
-  p.plan = plan;
-  p.plan_cnt = plan_cnt;
+  p.plan = w.plan;
+  p.plan_cnt = w.plan_cnt;
+  p.order = w.order;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  const Split sp = make_split(D, n_sm);
+  p.tiles_per_head = lf::tile_count(D);
+  p.n_whole = sp.n_whole;
+  p.pieces = sp.pieces;
+  p.part_o = w.part_o;
+  p.part_ml = w.part_ml;
   for (int i = 0; i < D.S; ++i) p.slots[i] = sink_slots[i];
   for (int i = 0; i < D.F; ++i) p.slots[D.S + i] = hist_slots[i];
-  if (D.d == 128) return D.B == 64 ? launch_attn_t<128, 64>(D, p, st) : launch_attn_t<128, 128>(D, p, st);
-  return D.B == 64 ? launch_attn_t<64, 64>(D, p, st) : launch_attn_t<64, 128>(D, p, st);
+  const int grid = sp.n_whole + sp.n_tail * sp.pieces;
+  if (D.d == 128)
+    rc = D.B == 64 ? launch_attn_t<128, 64>(D, p, grid, st) : launch_attn_t<128, 128>(D, p, grid, st);
+  else
+    rc = D.B == 64 ? launch_attn_t<64, 64>(D, p, grid, st) : launch_attn_t<64, 128>(D, p, grid, st);
+  if (rc != LF_OK || sp.n_tail == 0) return rc;
+  lf::merge_kernel<<<sp.n_tail, 256, 0, st>>>(p, D, D.d);
+  return cuda_status(cudaGetLastError());
 }
 
 // forward workspace carve-up
@@ -302,7 +370,9 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
   if (D.F > 0 && (block_idx == nullptr || !aligned(block_idx, 4))) return LF_ERR_INVALID_ARG;
   if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
   if ((rc = check_slots(sink_slots, D.S, D.n_slots)) != LF_OK) return rc;
-  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < attn_ws_bytes(D))
+  const size_t need = attn_ws_bytes(D);
+  if (need == 0) return LF_ERR_CUDA;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need)
     return LF_ERR_WORKSPACE;
   return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, block_idx,
                      out, lse, workspace, stream);
@@ -348,10 +418,19 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
                      lse, w.attn, stream);
 }
 
+int lf_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return LF_ERR_INVALID_ARG;
+  if (n == 0) return LF_OK;
+  lf::exp2_poly_kernel<<<lf::cdiv(n, 256), 256, 0, stream>>>(x, y, n);
+  return cuda_status(cudaGetLastError());
+}
+
 #ifdef LF_TRACE
-int lf_debug_set_trace(void* buf) {
+int lf_debug_set_trace(void* buf, void* cta_buf) {
   unsigned long long* p = static_cast<unsigned long long*>(buf);
-  return cudaMemcpyToSymbol(lf::g_lf_trace, &p, sizeof(p)) == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+  unsigned long long* q = static_cast<unsigned long long*>(cta_buf);
+  if (cudaMemcpyToSymbol(lf::g_lf_trace, &p, sizeof(p)) != cudaSuccess) return LF_ERR_CUDA;
+  return cudaMemcpyToSymbol(lf::g_lf_cta_trace, &q, sizeof(q)) == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 #endif
 

@@ -126,6 +126,65 @@ plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
 }
 
 // ---------------------------------------------------------------------------------
+// Launch order of the tiles: longest first (list scheduling by decreasing cost, so the
+// last CTAs to start are the cheapest).  Cost = key tiles = dense tiles + sparse tiles;
+// a counting sort over the sparse-tile count.  One CTA.  Tiles of equal cost keep an
+// arbitrary order, which changes no result.
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ order, const Dims D) {
+  __shared__ int hist[kMaxPlan + 1];
+  __shared__ int start[kMaxPlan + 1];
+  __shared__ int warp_tot[32];
+  const int ntot = tile_count(D) * D.H;
+  const int nb = kMaxPlan + 1;
+  for (int k = threadIdx.x; k < nb; k += blockDim.x) hist[k] = 0;
+  __syncthreads();
+  auto key = [&](int i) {
+    const int c = plan_cnt[i];
+    const int k = D.B == 64 ? (c + 1) / 2 : c;
+    return k < kMaxPlan ? k : kMaxPlan;
+  };
+  for (int i = threadIdx.x; i < ntot; i += blockDim.x) atomicAdd(&hist[key(i)], 1);
+  __syncthreads();
+  // exclusive scan in decreasing key order: start[k] = sum of hist[k'] for k' > k
+  const int per = (nb + blockDim.x - 1) / blockDim.x;     // buckets per thread (reversed)
+  int local = 0;
+  for (int q = 0; q < per; ++q) {
+    const int r = threadIdx.x * per + q;
+    if (r < nb) local += hist[kMaxPlan - r];
+  }
+  // block-wide exclusive scan of `local`
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = local;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += y;
+    }
+    warp_tot[lane] = v;                                  // inclusive over warps
+  }
+  __syncthreads();
+  int run = (w > 0 ? warp_tot[w - 1] : 0) + incl - local;
+  for (int q = 0; q < per; ++q) {
+    const int r = threadIdx.x * per + q;
+    if (r < nb) {
+      start[kMaxPlan - r] = run;
+      run += hist[kMaxPlan - r];
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < ntot; i += blockDim.x) order[atomicAdd(&start[key(i)], 1)] = i;
+}
+
+// ---------------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------------
 struct AttnParams {
@@ -136,8 +195,17 @@ struct AttnParams {
   CUtensorMap tm_vh;
   const uint32_t* plan;
   const int32_t* plan_cnt;
+  const int32_t* order;  // launch position -> tile (longest first)
   __nv_bfloat16* out;  // [ncur, H, d]
   float* lse;          // [H, ncur] or null
+  // work decomposition: CTAs [0, n_whole) take tiles whole; the remaining tiles (the last
+  // partial wave) are split into `pieces` key ranges each, written as partial softmax
+  // states to part_o / part_ml and combined by merge_kernel
+  int tiles_per_head;
+  int n_whole;
+  int pieces;
+  float* part_o;       // [n_tail * pieces, 128, d] unnormalised O
+  float* part_ml;      // [n_tail * pieces, 2, 128] row max (log2 units) and row sum
   int slots[LF_MAX_FRAMES];   // cache slot of frame position p (sinks, then history)
 };
 
@@ -184,6 +252,52 @@ constexpr int kSoftmaxWarps = 8;          // two warpgroups, alternate key tiles
 constexpr int kLaunchRegs = 168, kLowRegs = 72, kHighRegs = 216;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kAttnThreads * kLaunchRegs, "register split");
 
+// 2^x on the FMA pipe for x <= 8 (a share of the softmax exponentials is computed here
+// to unload the special-function unit).  Range reduction x = j + f, j = round(x),
+// f in [-1/2, 1/2], by adding and subtracting 1.5 * 2^23; 2^f by a degree-3 polynomial
+// (minimax relative error 7.5e-5, Remez fit, see gen_exp2_poly.py); j is added to the
+// IEEE-754 exponent field.  x is clamped at -126 so that the exponent field cannot go
+// below zero: -inf (a masked logit) gives about 1.2e-38.  Two lanes per instruction.
+constexpr float kExpC0 = 0.999928057f, kExpC1 = 0.693260968f, kExpC2 = 0.242611125f,
+                kExpC3 = 0.0551716685f, kShifter = 12582912.0f;
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = fadd2(x, make_float2(kShifter, kShifter));
+  const float2 j = fadd2(t, make_float2(-kShifter, -kShifter));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(make_float2(kExpC3, kExpC3), f, make_float2(kExpC2, kExpC2));
+  p = ffma2(p, f, make_float2(kExpC1, kExpC1));
+  p = ffma2(p, f, make_float2(kExpC0, kExpC0));
+  // bits(p) + (bits(t) << 23): the low bits of t hold j (two's complement)
+  return make_float2(__int_as_float(__float_as_int(p.x) + (int)((uint32_t)__float_as_int(t.x) * 8388608u)),
+                     __int_as_float(__float_as_int(p.y) + (int)((uint32_t)__float_as_int(t.y) * 8388608u)));
+}
+
+__device__ __forceinline__ float exp2_poly(float x) {
+  return exp2_poly2(make_float2(x, x)).x;
+}
+
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = exp2_poly(x[i]);
+}
+
+// How many of every 8 consecutive key pairs take the polynomial (tuning knob; 0 measured
+// fastest on B200 for this kernel, where the softmax is bound by its per-tile latency
+// chain rather than by the special-function unit).
+#ifndef LF_EXP2_FMA_PAIRS_OF_8
+#define LF_EXP2_FMA_PAIRS_OF_8 0
+#endif
+__host__ __device__ constexpr bool pair_on_fma(int e) {
+  return LF_EXP2_FMA_PAIRS_OF_8 == 0 ? false
+       : LF_EXP2_FMA_PAIRS_OF_8 == 1 ? (e & 7) == 5
+       : LF_EXP2_FMA_PAIRS_OF_8 == 2 ? ((e & 7) == 2 || (e & 7) == 6)
+       : LF_EXP2_FMA_PAIRS_OF_8 == 3 ? ((e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7)
+       : (e & 1) == 1;
+}
+
 template <int HD, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
@@ -198,8 +312,18 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x, h = blockIdx.y;
-  const int ntiles = gridDim.x;
+
+  // ---- work unit: a whole tile, or piece k of a tail tile
+  int pos, piece = -1, tail = 0;
+  if ((int)blockIdx.x < P.n_whole) {
+    pos = blockIdx.x;
+  } else {
+    tail = (blockIdx.x - P.n_whole) / P.pieces;
+    piece = (blockIdx.x - P.n_whole) % P.pieces;
+    pos = P.n_whole + tail;
+  }
+  const int tile = P.order[pos];
+  const int h = tile / P.tiles_per_head, t = tile % P.tiles_per_head;
 
   // query blocks of this tile
   const int qbA = BLK == 64 ? 2 * t : t;
@@ -207,10 +331,16 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   const int tokA = (qbA / D.nbpf) * D.T + (qbA % D.nbpf) * BLK;
   const int tokB = qbB >= 0 ? (qbB / D.nbpf) * D.T + (qbB % D.nbpf) * BLK : D.ncur;
 
-  const int cnt = P.plan_cnt[(size_t)h * ntiles + t];
+  const int cnt = P.plan_cnt[tile];
   const int n_dense = cdiv(D.ncur, 128);
   const int n_sparse = BLK == 64 ? cdiv(cnt, 2) : cnt;
-  const int n_iter = n_dense + n_sparse;
+  const int n_tile = n_dense + n_sparse;
+  // this CTA's key tiles: [j0, j0 + n_iter); local index l = j - j0 drives the pipeline
+  int j0 = 0, n_iter = n_tile;
+  if (piece >= 0) {
+    j0 = (int)((long long)piece * n_tile / P.pieces);
+    n_iter = (int)((long long)(piece + 1) * n_tile / P.pieces) - j0;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarQ], 1);
@@ -227,8 +357,13 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     tmem_alloc(s_tmem, L::kTmemCols);
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) {
+    LF_TR_CTA(0, smid());
+    LF_TR_CTA(1, globaltimer_ns());
+    LF_TR_CTA(3, n_iter);
+  }
   if (warp == 3) {
-    const uint32_t* src = P.plan + ((size_t)h * ntiles + t) * plan_stride(D);
+    const uint32_t* src = P.plan + (size_t)tile * plan_stride(D);
     for (int i = lane; i < cnt; i += 32) s_plan[i] = src[i];
   }
   if (warp == 0 && lane == 0) {
@@ -253,16 +388,17 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD + c * 64,
                   BLK == 64 ? tokB : tokA + 64);
     }
-    const int n_pos = 2 * n_iter + 1;               // V_{n-1} sits at position 2n
+    const int n_pos = 2 * n_iter + 1;               // V of the last tile sits at 2n
     int q = 0;
     for (; q < n_pos; ++q) {
       bool isK;
-      const int j = ring_tile(q, isK);
+      const int l = ring_tile(q, isK);
       const int slot = q % L::kSlots;
       const int rnd = q / L::kSlots;
-      if (isK && j >= n_iter) continue;            // no slot used, nothing to load
+      if (isK && l >= n_iter) continue;            // no slot used, nothing to load
       if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort)) break;
-      LF_TR(isK ? 0 : 1, j);
+      const int j = j0 + l;
+      LF_TR(isK ? 0 : 1, l);
       mbar_arrive_expect_tx(&full[slot], L::kStageBytes);
       uint8_t* st = smem + L::kRing + slot * L::kStageBytes;
       const CUtensorMap* tm_cur = isK ? &P.tm_kc : &P.tm_vc;
@@ -292,14 +428,14 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     // positions hold the only loads that nobody may have waited for)
     for (int x = max(0, q - L::kSlots); x < q; ++x) {
       bool isK;
-      const int jx = ring_tile(x, isK);
-      if (!(isK && jx >= n_iter)) mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1);
+      const int lx = ring_tile(x, isK);
+      if (!(isK && lx >= n_iter)) mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1);
     }
   }
   // -------------------------------------------------------------- MMA issuer
-  // Order: S0, S1, then for each i: PV_i (O_{i&1} += P_i V_i), S_{i+2} into the S buffer
-  // P_i was read from.  tcgen05.mma runs in issue order, so S_{i+2} overwrites P_i only
-  // after PV_i has consumed it, and the completion of S_{i+2} implies that of PV_i.
+  // Order: S0, S1, then for each l: PV_l (O_{l&1} += P_l V_l), S_{l+2} into the S buffer
+  // P_l was read from.  tcgen05.mma runs in issue order, so S_{l+2} overwrites P_l only
+  // after PV_l has consumed it, and the completion of S_{l+2} implies that of PV_l.
   else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, 0, 1);
@@ -307,12 +443,12 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     const uint32_t ring_base = smem_u32(smem + L::kRing);
     uint64_t* full = &bars[kBarRing];
     uint64_t* empty = &bars[kBarRing + L::kSlots];
-    auto issue_s = [&](int j) -> bool {
-      const int s = j & 1;
-      const int q = ring_pos_k(j), slot = q % L::kSlots;
-      LF_TR(2, j);
+    auto issue_s = [&](int l) -> bool {
+      const int s = l & 1;
+      const int q = ring_pos_k(l), slot = q % L::kSlots;
+      LF_TR(2, l);
       if (!mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort)) return false;
-      LF_TR(3, j);
+      LF_TR(3, l);
       tc_fence_after();
       const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
       const uint32_t k_addr = ring_base + slot * L::kStageBytes;
@@ -329,14 +465,14 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     bool ok = mbar_wait(&bars[kBarQ], 0, s_abort);
     if (ok) ok = issue_s(0);
     if (ok && n_iter > 1) ok = issue_s(1);
-    for (int i = 0; ok && i < n_iter; ++i) {
-      const int s = i & 1;
-      const int qv = ring_pos_v(i), vslot = qv % L::kSlots;
+    for (int l = 0; ok && l < n_iter; ++l) {
+      const int s = l & 1;
+      const int qv = ring_pos_v(l), vslot = qv % L::kSlots;
       ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort);
-      LF_TR(4, i);
-      if (ok) ok = mbar_wait(&bars[kBarPFull + s], (i >> 1) & 1, s_abort);
+      LF_TR(4, l);
+      if (ok) ok = mbar_wait(&bars[kBarPFull + s], (l >> 1) & 1, s_abort);
       if (!ok) break;
-      LF_TR(5, i);
+      LF_TR(5, l);
       tc_fence_after();
       const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
       const uint32_t o_tmem = tmem + (s ? L::kColO1 : L::kColO0);
@@ -345,9 +481,9 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
         mma_bf16_ts(o_tmem, p_tmem + ks * 8,
                     smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
                                     L::kRegion, 1024),
-                    idesc_pv, (i >= 2 || ks > 0) ? 1u : 0u);
+                    idesc_pv, (l >= 2 || ks > 0) ? 1u : 0u);
       mma_commit(&empty[vslot]);
-      if (i + 2 < n_iter) ok = issue_s(i + 2);
+      if (l + 2 < n_iter) ok = issue_s(l + 2);
     }
     // completion of everything issued: epilogue may read O, tensor memory may be freed
     mma_commit(&bars[kBarDone]);
@@ -356,7 +492,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   regs_inc<kHighRegs>();
   // -------------------------------------------------------------- softmax + epilogue
   {
-    const int wg = (warp - 4) >> 2;                        // handles key tiles j = wg, wg+2, ...
+    const int wg = (warp - 4) >> 2;                        // handles local tiles wg, wg+2, ...
     const int r = (threadIdx.x - 128) & 127;               // query row = TMEM lane
     const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t row_bit = (BLK == 64 && r >= 64) ? 2u : 1u;
@@ -366,10 +502,11 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int n_mine = 0;                                        // PVs into this group's O
-    for (int j = wg; j < n_iter; j += 2, ++n_mine) {
-      if (threadIdx.x == 128) LF_TR(6, j);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + wg], (j >> 1) & 1, s_abort)) && ok;
-      if (threadIdx.x == 128) LF_TR(7, j);
+    for (int l = wg; l < n_iter; l += 2, ++n_mine) {
+      const int j = j0 + l;
+      if (threadIdx.x == 128) LF_TR(6, l);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + wg], (l >> 1) & 1, s_abort)) && ok;
+      if (threadIdx.x == 128) LF_TR(7, l);
       tc_fence_after();
       float sv[128];
 #pragma unroll
@@ -377,7 +514,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       tmem_ld_wait();
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) reg_fence32(sv + ch * 32);
-      if (threadIdx.x == 128) LF_TR(8, j);
+      if (threadIdx.x == 128) LF_TR(8, l);
 
       // valid key columns of this row: [0, v0) and [64, 64 + v1)
       int v0, v1;
@@ -425,7 +562,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       float m_new = m_run;
       bool resc = false;
       if (m_tile > m_run + 8.0f) { m_new = m_tile; resc = true; }
-      // lazy rescale of this group's O: its previous PV (PV_{j-2}) completed before S_j did
+      // lazy rescale of this group's O: its previous PV (PV_{l-2}) completed before S_l did
       if (n_mine > 0 && __any_sync(0xffffffffu, resc)) {
         const float a = resc ? exp2f(m_run - m_new) : 1.f;
 #pragma unroll
@@ -440,30 +577,40 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
         }
         if (resc) l_run *= a;
       }
-      if (threadIdx.x == 128) LF_TR(9, j);
+      if (threadIdx.x == 128) LF_TR(9, l);
       const float mref = (m_new == -INFINITY) ? 0.f : m_new;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
+      float2 ps0 = make_float2(0.f, 0.f), ps1 = make_float2(0.f, 0.f);
+      // probabilities in four chunks of 32 keys; each chunk is packed to bf16 pairs and
+      // stored to tensor memory (16 columns) at once, which bounds register pressure
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float pk[32];
+      for (int ch = 0; ch < 4; ++ch) {
+        float pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2_approx(fmaf(sv[half * 64 + 2 * e], c, -mref));
-          const float p1 = ex2_approx(fmaf(sv[half * 64 + 2 * e + 1], c, -mref));
-          ps[e & 3] += p0 + p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+        for (int e = 0; e < 16; ++e) {
+          const int i0 = ch * 32 + 2 * e;
+          const float2 x = ffma2(make_float2(sv[i0], sv[i0 + 1]), c2, nm2);
+          float2 p;
+          if (pair_on_fma(ch * 16 + e)) {
+            p = exp2_poly2(x);
+          } else {
+            p.x = ex2_approx(x.x);
+            p.y = ex2_approx(x.y);
+          }
+          if (e & 1) ps1 = fadd2(ps1, p); else ps0 = fadd2(ps0, p);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
           pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&b2));
         }
-        tmem_st32(t_row + s_col + half * 32, pk);
+        tmem_st16(t_row + s_col + ch * 16, pk);
       }
-      if (threadIdx.x == 128) LF_TR(10, j);
+      if (threadIdx.x == 128) LF_TR(10, l);
       tmem_st_wait();
-      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      l_run += (ps0.x + ps0.y) + (ps1.x + ps1.y);
       m_run = m_new;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarPFull + wg]);
-      if (threadIdx.x == 128) LF_TR(11, j);
+      if (threadIdx.x == 128) LF_TR(11, l);
     }
     ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0, s_abort)) && ok;
     // merge the two groups' partial softmax states: O = sum_w 2^(m_w - m) O_w / l
@@ -482,10 +629,13 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       else { qb = qbA; i = r; }
       const bool valid = qb >= 0 && i < block_len(D, qb % D.nbpf);
       const int tok = qb >= 0 ? (qb / D.nbpf) * D.T + (qb % D.nbpf) * BLK + i : 0;
-      const float inv_l = 1.0f / l_tot;
+      // a whole tile is normalised here; a piece keeps sum_w 2^(m_w - m) O_w, m and l
+      const float inv_l = piece < 0 ? 1.0f / l_tot : 1.0f;
       // this group writes output columns [wg*HD/2, (wg+1)*HD/2) from both accumulators
       const float w0 = (wg == 0 ? w_me : w_o) * inv_l, w1 = (wg == 0 ? w_o : w_me) * inv_l;
+      const int unit = tail * P.pieces + piece;
       __nv_bfloat16* orow = P.out + ((size_t)tok * D.H + h) * HD + wg * (HD / 2);
+      float* prow = P.part_o + ((size_t)unit * 128 + r) * HD + wg * (HD / 2);
 #pragma unroll
       for (int ch = 0; ch < HD / 64; ++ch) {
         float a[32], b[32];
@@ -495,36 +645,93 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
         tmem_ld_wait();
         reg_fence32(a);
         reg_fence32(b);
-        if (valid) {
-          uint32_t pw[16];
+        float x[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            // a group that never accumulated has weight 0 and its O is not read into the sum
-            const float x0 = (w0 > 0.f ? a[2 * e] * w0 : 0.f) + (w1 > 0.f ? b[2 * e] * w1 : 0.f);
-            const float x1 = (w0 > 0.f ? a[2 * e + 1] * w0 : 0.f) +
-                             (w1 > 0.f ? b[2 * e + 1] * w1 : 0.f);
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
-            pw[e] = *reinterpret_cast<uint32_t*>(&b2);
+        for (int e = 0; e < 32; ++e)
+          // a group that never accumulated has weight 0 and its O is not read into the sum
+          x[e] = (w0 > 0.f ? a[e] * w0 : 0.f) + (w1 > 0.f ? b[e] * w1 : 0.f);
+        if (piece < 0) {
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint32_t pw[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(x[8 * e + 2 * k], x[8 * e + 2 * k + 1]);
+                pw[k] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              dst[e] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            }
           }
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(prow + ch * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pw[4 * e], pw[4 * e + 1], pw[4 * e + 2], pw[4 * e + 3]);
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
         }
       }
-      if (valid && wg == 0 && P.lse != nullptr)
-        P.lse[(size_t)h * D.ncur + tok] = (m_all + log2f(l_tot)) * 0.6931471805599453f;
+      if (piece < 0) {
+        if (valid && wg == 0 && P.lse != nullptr)
+          P.lse[(size_t)h * D.ncur + tok] = (m_all + log2f(l_tot)) * 0.6931471805599453f;
+      } else if (wg == 0) {
+        P.part_ml[((size_t)unit * 2) * 128 + r] = m_all;
+        P.part_ml[((size_t)unit * 2 + 1) * 128 + r] = l_tot;
+      }
       tc_fence_before();
     }
   }
   }
   __syncthreads();
+  if (threadIdx.x == 0) LF_TR_CTA(2, globaltimer_ns());
   if (warp == 1) {
     // everything the MMA thread issued is complete before tensor memory is released
     if (lane == 0) mbar_wait_drain(&bars[kBarDone], 0);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// Combines the partial softmax states of the pieces of each tail tile (fixed order):
+// m = max_k m_k, l = sum_k 2^(m_k - m) l_k, O = sum_k 2^(m_k - m) O_k / l.
+// One CTA per tail tile, one thread per (row, 4 channels).
+__global__ void __launch_bounds__(256)
+merge_kernel(const AttnParams P, const Dims D, int HD) {
+  const int tail = blockIdx.x;
+  const int tile = P.order[P.n_whole + tail];
+  const int h = tile / P.tiles_per_head, t = tile % P.tiles_per_head;
+  const int qbA = D.B == 64 ? 2 * t : t;
+  const int qbB = (D.B == 64 && 2 * t + 1 < D.nqb) ? 2 * t + 1 : -1;
+  const int c4n = HD / 4;
+  for (int idx = threadIdx.x; idx < 128 * c4n; idx += blockDim.x) {
+    const int r = idx / c4n, c4 = idx % c4n;
+    int qb, i;
+    if (D.B == 64) { qb = r < 64 ? qbA : qbB; i = r & 63; }
+    else { qb = qbA; i = r; }
+    if (qb < 0 || i >= block_len(D, qb % D.nbpf)) continue;
+    const int tok = (qb / D.nbpf) * D.T + (qb % D.nbpf) * D.B + i;
+    float m = -INFINITY;
+    for (int k = 0; k < P.pieces; ++k)
+      m = fmaxf(m, P.part_ml[((size_t)(tail * P.pieces + k) * 2) * 128 + r]);
+    float l = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < P.pieces; ++k) {
+      const int unit = tail * P.pieces + k;
+      const float mk = P.part_ml[((size_t)unit * 2) * 128 + r];
+      if (mk == -INFINITY) continue;
+      const float w = exp2f(mk - m);
+      l += w * P.part_ml[((size_t)unit * 2 + 1) * 128 + r];
+      const float4 x = reinterpret_cast<const float4*>(P.part_o + ((size_t)unit * 128 + r) * HD)[c4];
+      o.x += w * x.x; o.y += w * x.y; o.z += w * x.z; o.w += w * x.w;
+    }
+    const float inv = 1.0f / l;
+    __nv_bfloat162 a = __floats2bfloat162_rn(o.x * inv, o.y * inv);
+    __nv_bfloat162 b = __floats2bfloat162_rn(o.z * inv, o.w * inv);
+    uint2 pk = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+    reinterpret_cast<uint2*>(P.out + ((size_t)tok * D.H + h) * HD)[c4] = pk;
+    if (c4 == 0 && P.lse != nullptr)
+      P.lse[(size_t)h * D.ncur + tok] = (m + log2f(l)) * 0.6931471805599453f;
   }
 }
 

@@ -43,6 +43,11 @@ __device__ __forceinline__ void record_status(int code) {
 #ifdef LF_TRACE
 __device__ unsigned long long* g_lf_trace = nullptr;
 constexpr int kTraceCtas = 4, kTraceEvents = 16, kTraceIters = 256;
+__device__ unsigned long long* g_lf_cta_trace = nullptr;   // [cta][4]: smid, t0, t1, iters
+#define LF_TR_CTA(k, v)                                                                  \
+  do {                                                                                   \
+    if (g_lf_cta_trace) g_lf_cta_trace[(size_t)(blockIdx.x + blockIdx.y * gridDim.x) * 4 + (k)] = (v); \
+  } while (0)
 #define LF_TR(ev, it)                                                                    \
   do {                                                                                   \
     const int _cta = blockIdx.x + blockIdx.y * gridDim.x;                                \
@@ -52,7 +57,14 @@ constexpr int kTraceCtas = 4, kTraceEvents = 16, kTraceIters = 256;
   } while (0)
 #else
 #define LF_TR(ev, it) do {} while (0)
+#define LF_TR_CTA(k, v) do {} while (0)
 #endif
+
+__device__ __forceinline__ uint32_t smid() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return r;
+}
 
 // ------------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -133,6 +145,26 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// Packed fp32 pair arithmetic (sm_100 f32x2 instructions): one instruction, two lanes.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, C, D;\n\t"
+      "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\tmov.b64 C, {%6, %7};\n\t"
+      "fma.rn.f32x2 D, A, B, C;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\t"
+      "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "add.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32; 2^-inf = 0).
@@ -260,6 +292,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
         "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
         "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
         "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 

@@ -146,6 +146,12 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
                      void* workspace, size_t workspace_bytes, void* out, float* lse,
                      int32_t* block_idx_out, cudaStream_t stream);
 
+/* Test hook, not part of the attention path: evaluates the FMA-pipe exponential the
+ * attention softmax uses for part of its probabilities, y[i] = 2^x[i] for x[i] <= 8
+ * (degree-3 polynomial after round-to-nearest range reduction; relative error below
+ * 1e-4 for -125 <= x <= 8; x below -126 gives about 1.2e-38).  x, y: device fp32 [n]. */
+int lf_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+
 /* Reads (synchronising the current device) and optionally clears the device status word
  * of the current device: LF_OK, LF_ERR_BAD_INDEX or LF_ERR_TIMEOUT.  Returns LF_ERR_CUDA
  * if the read itself fails. */
