@@ -63,6 +63,14 @@ def executed_flops(shape, block_idx_np) -> int:
     return int(4 * shape.d * (qlen[None, :] * (dense + sel)).sum())
 
 
+def tail_split(shape, n_sm=148) -> bool:
+    """Whether the attention launch splits its last, partial wave of tiles (mirrors the
+    library's rule: the last wave is less than half full)."""
+    tiles = shape.H * (-(-shape.n_cur_frames * -(-shape.T // shape.block) // (2 if shape.block == 64 else 1)))
+    r = tiles % n_sm
+    return r != 0 and 2 * r <= n_sm
+
+
 def selection_bytes(shape) -> int:
     return 2 * shape.H * shape.d * shape.T * (shape.n_cur_frames + shape.n_hist)
 
@@ -255,7 +263,8 @@ def run_lf(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     flops = executed_flops(sh, bidx.cpu().numpy())
-    launches_per_step = 6 if sh.n_hist > 0 else 2
+    # pool_blocks, pool_frames, select_frames, select_blocks | plan, schedule, attn (+ merge)
+    launches_per_step = (4 if sh.n_hist > 0 else 0) + 3 + (1 if tail_split(sh) else 0)
 
     clocks = ClockSampler(local_rank)
     clocks.start()

@@ -62,6 +62,8 @@ int check_slots(const int32_t* slots, int n, int n_slots) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? LF_OK : LF_ERR_CUDA; }
 
+constexpr size_t kMaxSmem = 227 * 1024;   // opt-in shared memory per block on sm_100
+
 // --------------------------------------------------------------- tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -114,6 +116,7 @@ int launch_compress(const Dims& D, const void* q, const void* k_cache, const int
 int launch_select_frames(const Dims& D, const float* q_blk, const float* k_frm,
                          int32_t* frame_idx, float* frame_score, cudaStream_t st) {
   const size_t smem = ((size_t)D.F * (D.d + 4) + (size_t)lf::kSelWarps * D.d) * sizeof(float);
+  if (smem > kMaxSmem) return LF_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(lf::select_frames_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return LF_ERR_CUDA;
@@ -126,7 +129,9 @@ int launch_select_frames(const Dims& D, const float* q_blk, const float* k_frm,
 int launch_select_blocks(const Dims& D, const float* q_blk, const float* k_blk,
                          const int32_t* frame_idx, int32_t* block_idx, float* block_score,
                          cudaStream_t st) {
-  const size_t smem = ((size_t)D.nbpf * (D.d + 4) + (size_t)lf::kSelWarps * D.d) * sizeof(float);
+  const size_t smem = ((size_t)D.nbpf * (D.d + 4) + (size_t)lf::kSelBatch * D.d) * sizeof(float) +
+                      (size_t)D.nqb * sizeof(int);
+  if (smem > kMaxSmem) return LF_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(lf::select_blocks_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return LF_ERR_CUDA;

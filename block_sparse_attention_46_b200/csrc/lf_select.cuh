@@ -129,8 +129,19 @@ constexpr int kMaxPerLane = 8;   // candidates per lane: up to 256 frames or blo
 
 // Selects the k best of n candidates held lane-strided (candidate c = lane + 32*j lives
 // in sc[j] of lane c%32).  Returns in `taken` (bit j per lane) the chosen candidates.
+// n <= 32: each lane counts the candidates better than its own (its rank) in one sweep
+// of shuffles; larger n: k rounds of warp argmax.
 __device__ __forceinline__ uint32_t warp_topk(const float* sc, int n, int k) {
   const int lane = threadIdx.x & 31;
+  if (n <= 32) {
+    int rank = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float sj = __shfl_sync(0xffffffffu, sc[0], j);
+      rank += (j < n && better(sj, j, sc[0], lane)) ? 1 : 0;
+    }
+    return (lane < n && rank < k) ? 1u : 0u;
+  }
   uint32_t taken = 0;
   for (int r = 0; r < k; ++r) {
     float bs = -INFINITY;
@@ -158,6 +169,17 @@ __device__ __forceinline__ void warp_write_ascending(uint32_t taken, int n, int3
     if ((taken >> j) & 1u) out[before + __popc(m & ((1u << lane) - 1u))] = id_base + lane + 32 * j;
     before += __popc(m);
   }
+}
+
+// q . k over d channels in a fixed order (four interleaved partial sums, then combined).
+__device__ __forceinline__ float dot_fixed(const float* q, const float* k, int d) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  for (int c = 0; c < d; c += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(q + c);
+    const float4 y = *reinterpret_cast<const float4*>(k + c);
+    a0 = fmaf(x.x, y.x, a0); a1 = fmaf(x.y, y.y, a1); a2 = fmaf(x.z, y.z, a2); a3 = fmaf(x.w, y.w, a3);
+  }
+  return (a0 + a1) + (a2 + a3);
 }
 
 // ---------------------------------------------------------------------------------
@@ -197,13 +219,7 @@ select_frames_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
     const int f = lane + 32 * j;
     float s = -INFINITY;
     if (f < D.F) {
-      const float* kv = sk + (size_t)f * pitch;
-      s = 0.f;
-      for (int c = 0; c < D.d; c += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(qv + c);
-        const float4 b = *reinterpret_cast<const float4*>(kv + c);
-        s = fmaf(a.x, b.x, s); s = fmaf(a.y, b.y, s); s = fmaf(a.z, b.z, s); s = fmaf(a.w, b.w, s);
-      }
+      s = dot_fixed(qv, sk + (size_t)f * pitch, D.d);
       if (frame_score) frame_score[((size_t)h * D.nqb + qb) * D.F + f] = s;
     }
     sc[j] = s;
@@ -214,11 +230,14 @@ select_frames_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
 
 // ---------------------------------------------------------------------------------
 // (c) Block selection inside chosen frames.  CTA = (history frame f, head h): k_blk[h, f]
-// is staged in shared memory once; each warp walks the query blocks of head h whose
-// chosen-frame list holds f (at rank j), scores the frame's blocks (lane c: blocks c,
+// is staged in shared memory once, and the query blocks of head h whose chosen-frame list
+// holds f (at rank j) are listed first; then, in batches whose pooled queries are staged
+// in shared memory, a warp per query block scores the frame's blocks (lane c: blocks c,
 // c+32, ...), keeps the kb best and writes them, ascending, to slots [j*kb, (j+1)*kb) of
 // block_idx[h, qb] — ascending overall because the frame list is ascending.
 // ---------------------------------------------------------------------------------
+constexpr int kSelBatch = 32;
+
 __global__ void __launch_bounds__(kSelWarps * 32)
 select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_blk,
                      const int32_t* __restrict__ frame_idx, int32_t* __restrict__ block_idx,
@@ -227,59 +246,67 @@ select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
   float* sk = reinterpret_cast<float*>(sm4);
   const int f = blockIdx.x, h = blockIdx.y;
   const int pitch = D.d + 4;
-  float* sq = sk + (size_t)D.nbpf * pitch;            // [kSelWarps][d]
+  float* sq = sk + (size_t)D.nbpf * pitch;            // [kSelBatch][d]
+  int* s_list = reinterpret_cast<int*>(sq + (size_t)kSelBatch * D.d);   // [nqb] packed qb | rank
+  __shared__ int s_n;
+  if (threadIdx.x == 0) s_n = 0;
   for (int i = threadIdx.x; i < D.nbpf * (D.d / 4); i += blockDim.x) {
     const int b = i / (D.d / 4), c4 = i % (D.d / 4);
     reinterpret_cast<float4*>(sk + (size_t)b * pitch)[c4] =
         reinterpret_cast<const float4*>(k_blk + (((size_t)h * D.F + f) * D.nbpf + b) * D.d)[c4];
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* qv = sq + warp * D.d;
-  for (int qb = warp; qb < D.nqb; qb += kSelWarps) {
+  // which query blocks chose frame f, and at which rank (lists validated on the way)
+  for (int qb = threadIdx.x; qb < D.nqb; qb += blockDim.x) {
     const int32_t* fl = frame_idx + ((size_t)h * D.nqb + qb) * D.kf;
-    // rank of f in the (ascending) chosen list; validate the list on the way
     int rank = -1;
     bool bad = false;
-    for (int j = lane; j < D.kf; j += 32) {
+    int prev = -1;
+    for (int j = 0; j < D.kf; ++j) {
       const int v = fl[j];
-      if (v < 0 || v >= D.F || (j > 0 && fl[j - 1] >= v)) bad = true;
+      bad |= v < 0 || v >= D.F || v <= prev;
+      prev = v;
       if (v == f) rank = j;
     }
-    bad = __any_sync(0xffffffffu, bad);
-    rank = __reduce_max_sync(0xffffffffu, rank);
     if (bad) {
-      if (lane == 0 && f == 0) record_status(LF_ERR_BAD_INDEX);
-      continue;
+      if (f == 0) record_status(LF_ERR_BAD_INDEX);
+    } else if (rank >= 0) {
+      s_list[atomicAdd(&s_n, 1)] = (qb << 10) | rank;
     }
-    if (rank < 0) continue;
-    for (int c4 = lane; c4 < D.d / 4; c4 += 32)
-      reinterpret_cast<float4*>(qv)[c4] =
+  }
+  __syncthreads();
+  const int n = s_n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int b0 = 0; b0 < n; b0 += kSelBatch) {
+    const int nb = min(kSelBatch, n - b0);
+    for (int i = threadIdx.x; i < nb * (D.d / 4); i += blockDim.x) {
+      const int e = i / (D.d / 4), c4 = i % (D.d / 4);
+      const int qb = s_list[b0 + e] >> 10;
+      reinterpret_cast<float4*>(sq + (size_t)e * D.d)[c4] =
           reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + qb) * D.d)[c4];
-    __syncwarp();
-    float sc[kMaxPerLane];
-#pragma unroll
-    for (int j = 0; j < kMaxPerLane; ++j) {
-      const int b = lane + 32 * j;
-      float s = -INFINITY;
-      if (b < D.nbpf) {
-        const float* kv = sk + (size_t)b * pitch;
-        s = 0.f;
-        for (int c = 0; c < D.d; c += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(qv + c);
-          const float4 y = *reinterpret_cast<const float4*>(kv + c);
-          s = fmaf(x.x, y.x, s); s = fmaf(x.y, y.y, s); s = fmaf(x.z, y.z, s); s = fmaf(x.w, y.w, s);
-        }
-        if (block_score)
-          block_score[(((size_t)h * D.nqb + qb) * D.kf + rank) * D.nbpf + b] = s;
-      }
-      sc[j] = s;
     }
-    const uint32_t taken = warp_topk(sc, D.nbpf, D.kb);
-    warp_write_ascending(taken, D.nbpf,
-                         block_idx + ((size_t)h * D.nqb + qb) * D.nsel + (size_t)rank * D.kb,
-                         f * D.nbpf);
-    __syncwarp();
+    __syncthreads();
+    for (int e = warp; e < nb; e += kSelWarps) {
+      const int qb = s_list[b0 + e] >> 10, rank = s_list[b0 + e] & 1023;
+      const float* qv = sq + (size_t)e * D.d;
+      float sc[kMaxPerLane];
+#pragma unroll
+      for (int j = 0; j < kMaxPerLane; ++j) {
+        const int b = lane + 32 * j;
+        float sres = -INFINITY;
+        if (b < D.nbpf) {
+          sres = dot_fixed(qv, sk + (size_t)b * pitch, D.d);
+          if (block_score)
+            block_score[(((size_t)h * D.nqb + qb) * D.kf + rank) * D.nbpf + b] = sres;
+        }
+        sc[j] = sres;
+      }
+      const uint32_t taken = warp_topk(sc, D.nbpf, D.kb);
+      warp_write_ascending(taken, D.nbpf,
+                           block_idx + ((size_t)h * D.nqb + qb) * D.nsel + (size_t)rank * D.kb,
+                           f * D.nbpf);
+    }
+    __syncthreads();
   }
 }
 
