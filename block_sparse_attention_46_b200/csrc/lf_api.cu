@@ -130,7 +130,7 @@ int launch_select_blocks(const Dims& D, const float* q_blk, const float* k_blk,
                          const int32_t* frame_idx, int32_t* block_idx, float* block_score,
                          cudaStream_t st) {
   const size_t smem = ((size_t)D.nbpf * (D.d + 4) + (size_t)lf::kSelBatch * D.d) * sizeof(float) +
-                      (size_t)D.nqb * sizeof(int);
+                      (size_t)D.nqb * (1 + D.kf) * sizeof(int);
   if (smem > kMaxSmem) return LF_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(lf::select_blocks_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -261,7 +261,7 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   else
     rc = D.B == 64 ? launch_attn_t<64, 64>(D, p, grid, st) : launch_attn_t<64, 128>(D, p, grid, st);
   if (rc != LF_OK || sp.n_tail == 0) return rc;
-  lf::merge_kernel<<<sp.n_tail, 256, 0, st>>>(p, D, D.d);
+  lf::merge_kernel<<<dim3(sp.n_tail, 128 / lf::kMergeRows), 256, 0, st>>>(p, D, D.d);
   return cuda_status(cudaGetLastError());
 }
 

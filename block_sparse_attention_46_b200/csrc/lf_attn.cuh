@@ -233,7 +233,8 @@ struct AttnLayout {
 };
 
 // barrier indices: ring full/empty barriers follow these
-enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 5, kBarRing = 6 };
+// P barriers: kBarPFull + 2 * buffer + half (keys 0-63, 64-127)
+enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 7, kBarRing = 8 };
 
 // position of a tile in the ring's load order: K0, K1, V0, K2, V1, K3, V2, ...
 __device__ __forceinline__ int ring_pos_k(int j) { return j < 2 ? j : 2 * j - 1; }
@@ -346,7 +347,8 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     mbar_init(&bars[kBarQ], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kBarSFull + s], 1);
-      mbar_init(&bars[kBarPFull + s], 4);
+      mbar_init(&bars[kBarPFull + 2 * s], 4);
+      mbar_init(&bars[kBarPFull + 2 * s + 1], 4);
     }
     for (int q = 0; q < 2 * L::kSlots; ++q) mbar_init(&bars[kBarRing + q], 1);
     mbar_init(&bars[kBarDone], 1);
@@ -470,18 +472,25 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       const int qv = ring_pos_v(l), vslot = qv % L::kSlots;
       ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort);
       LF_TR(4, l);
-      if (ok) ok = mbar_wait(&bars[kBarPFull + s], (l >> 1) & 1, s_abort);
-      if (!ok) break;
-      LF_TR(5, l);
-      tc_fence_after();
       const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
       const uint32_t o_tmem = tmem + (s ? L::kColO1 : L::kColO0);
+      // P arrives in two halves (keys 0-63, 64-127); each half's four MMAs go as soon
+      // as it is written
+      for (int hf = 0; ok && hf < 2; ++hf) {
+        ok = mbar_wait(&bars[kBarPFull + 2 * s + hf], (l >> 1) & 1, s_abort);
+        if (!ok) break;
+        if (hf == 0) LF_TR(5, l);
+        tc_fence_after();
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)            // 128 keys, 16 per MMA, 8 columns each
-        mma_bf16_ts(o_tmem, p_tmem + ks * 8,
-                    smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
-                                    L::kRegion, 1024),
-                    idesc_pv, (l >= 2 || ks > 0) ? 1u : 0u);
+        for (int k4 = 0; k4 < 4; ++k4) {        // 16 keys per MMA, 8 P columns each
+          const int ks = hf * 4 + k4;
+          mma_bf16_ts(o_tmem, p_tmem + ks * 8,
+                      smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
+                                      L::kRegion, 1024),
+                      idesc_pv, (l >= 2 || ks > 0) ? 1u : 0u);
+        }
+      }
+      if (!ok) break;
       mma_commit(&empty[vslot]);
       if (l + 2 < n_iter) ok = issue_s(l + 2);
     }
@@ -581,35 +590,47 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       const float mref = (m_new == -INFINITY) ? 0.f : m_new;
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
       float2 ps0 = make_float2(0.f, 0.f), ps1 = make_float2(0.f, 0.f);
-      // probabilities in four chunks of 32 keys; each chunk is packed to bf16 pairs and
-      // stored to tensor memory (16 columns) at once, which bounds register pressure
+      // probabilities per 64-key half (published separately so that the PV MMAs of the
+      // first half overlap the exponentials of the second), in chunks of 32 keys packed to
+      // bf16 pairs and stored to tensor memory (16 columns) at once.  A half with no valid
+      // key for this row (warp-uniform) is written as zeros without exponentials.
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        float pk[16];
+      for (int hf = 0; hf < 2; ++hf) {
+        const bool any = (hf == 0 ? v0 : v1) > 0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i0 = ch * 32 + 2 * e;
-          const float2 x = ffma2(make_float2(sv[i0], sv[i0 + 1]), c2, nm2);
-          float2 p;
-          if (pair_on_fma(ch * 16 + e)) {
-            p = exp2_poly2(x);
+        for (int cc = 0; cc < 2; ++cc) {
+          const int ch = hf * 2 + cc;
+          float pk[16];
+          if (any) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int i0 = ch * 32 + 2 * e;
+              const float2 x = ffma2(make_float2(sv[i0], sv[i0 + 1]), c2, nm2);
+              float2 p;
+              if (pair_on_fma(ch * 16 + e)) {
+                p = exp2_poly2(x);
+              } else {
+                p.x = ex2_approx(x.x);
+                p.y = ex2_approx(x.y);
+              }
+              if (e & 1) ps1 = fadd2(ps1, p); else ps0 = fadd2(ps0, p);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
+              pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&b2));
+            }
           } else {
-            p.x = ex2_approx(x.x);
-            p.y = ex2_approx(x.y);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = 0.f;
           }
-          if (e & 1) ps1 = fadd2(ps1, p); else ps0 = fadd2(ps0, p);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
-          pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&b2));
+          tmem_st16(t_row + s_col + ch * 16, pk);
         }
-        tmem_st16(t_row + s_col + ch * 16, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarPFull + 2 * wg + hf]);
       }
       if (threadIdx.x == 128) LF_TR(10, l);
-      tmem_st_wait();
       l_run += (ps0.x + ps0.y) + (ps1.x + ps1.y);
       m_run = m_new;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarPFull + wg]);
       if (threadIdx.x == 128) LF_TR(11, l);
     }
     ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0, s_abort)) && ok;
@@ -695,7 +716,9 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
 
 // Combines the partial softmax states of the pieces of each tail tile (fixed order):
 // m = max_k m_k, l = sum_k 2^(m_k - m) l_k, O = sum_k 2^(m_k - m) O_k / l.
-// One CTA per tail tile, one thread per (row, 4 channels).
+// CTA = (tail tile, group of kMergeRows rows); one thread per (row, 4 channels).
+constexpr int kMergeRows = 8;
+
 __global__ void __launch_bounds__(256)
 merge_kernel(const AttnParams P, const Dims D, int HD) {
   const int tail = blockIdx.x;
@@ -704,8 +727,8 @@ merge_kernel(const AttnParams P, const Dims D, int HD) {
   const int qbA = D.B == 64 ? 2 * t : t;
   const int qbB = (D.B == 64 && 2 * t + 1 < D.nqb) ? 2 * t + 1 : -1;
   const int c4n = HD / 4;
-  for (int idx = threadIdx.x; idx < 128 * c4n; idx += blockDim.x) {
-    const int r = idx / c4n, c4 = idx % c4n;
+  for (int idx = threadIdx.x; idx < kMergeRows * c4n; idx += blockDim.x) {
+    const int r = blockIdx.y * kMergeRows + idx / c4n, c4 = idx % c4n;
     int qb, i;
     if (D.B == 64) { qb = r < 64 ? qbA : qbB; i = r & 63; }
     else { qb = qbA; i = r; }

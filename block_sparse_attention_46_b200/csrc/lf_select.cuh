@@ -103,7 +103,15 @@ __global__ void pool_frames_kernel(const float* __restrict__ k_blk, float* __res
   const float invT = 1.0f / (float)D.T;
   for (int c = threadIdx.x; c < D.d; c += blockDim.x) {
     float s = 0.f;
-    for (int b = 0; b < D.nbpf; ++b) s += (float)block_len(D, b) * src[(size_t)b * D.d + c];
+    int b = 0;
+    for (; b + 8 <= D.nbpf; b += 8) {          // eight loads in flight, summed in block order
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = src[(size_t)(b + u) * D.d + c];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s += (float)block_len(D, b + u) * v[u];
+    }
+    for (; b < D.nbpf; ++b) s += (float)block_len(D, b) * src[(size_t)b * D.d + c];
     k_frm[((size_t)h * D.F + f) * D.d + c] = s * invT;
   }
 }
@@ -248,6 +256,7 @@ select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
   const int pitch = D.d + 4;
   float* sq = sk + (size_t)D.nbpf * pitch;            // [kSelBatch][d]
   int* s_list = reinterpret_cast<int*>(sq + (size_t)kSelBatch * D.d);   // [nqb] packed qb | rank
+  int* s_fl = s_list + D.nqb;                                             // [nqb * kf] frame lists
   __shared__ int s_n;
   if (threadIdx.x == 0) s_n = 0;
   for (int i = threadIdx.x; i < D.nbpf * (D.d / 4); i += blockDim.x) {
@@ -255,10 +264,12 @@ select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
     reinterpret_cast<float4*>(sk + (size_t)b * pitch)[c4] =
         reinterpret_cast<const float4*>(k_blk + (((size_t)h * D.F + f) * D.nbpf + b) * D.d)[c4];
   }
+  for (int i = threadIdx.x; i < D.nqb * D.kf; i += blockDim.x)
+    s_fl[i] = frame_idx[(size_t)h * D.nqb * D.kf + i];
   __syncthreads();
   // which query blocks chose frame f, and at which rank (lists validated on the way)
   for (int qb = threadIdx.x; qb < D.nqb; qb += blockDim.x) {
-    const int32_t* fl = frame_idx + ((size_t)h * D.nqb + qb) * D.kf;
+    const int* fl = s_fl + (size_t)qb * D.kf;
     int rank = -1;
     bool bad = false;
     int prev = -1;
