@@ -71,6 +71,22 @@ def tail_split(shape, n_sm=148) -> bool:
     return r != 0 and 2 * r <= n_sm
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest value of x over all ranks (the job's time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job TFLOP/s: every rank processed its own chunk in at most `ms`."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def selection_bytes(shape) -> int:
     return 2 * shape.H * shape.d * shape.T * (shape.n_cur_frames + shape.n_hist)
 
@@ -287,13 +303,9 @@ def run_lf(args, rank, world, local_rank):
     assert lf.lf_device_status() == 0, "device status reported an error"
 
     step_ms = [a + b for a, b in zip(sel_ms, att_ms)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_step = total_ms / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = weak_scaling_value(flops, world, ms_step)
 
     # e2e through lf_forward_chunk with host buffers
     hq = {k: t[k].cpu().pin_memory() for k in ("q", "k_cur", "v_cur")}
@@ -326,11 +338,7 @@ def run_lf(args, rank, world, local_rank):
         g_e2e.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
     h2d = sum(hq[k].numel() * hq[k].element_size() for k in hq)
     d2h = hout.numel() * hout.element_size()
 
@@ -357,7 +365,7 @@ def run_lf(args, rank, world, local_rank):
                                "unit": "GB/s", "frac": sel_gbs / pk["hbm_gbs"],
                                "kernels": "pool_blocks + pool_frames + select_frames + select_blocks",
                                "peak_source": f"{src} hbm_gbs"},
-        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": weak_scaling_value(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "lf_forward_chunk (replayed as one CUDA graph with the copies)"},
         "gpu_launches": launches_per_step * args.steps,

@@ -1,0 +1,51 @@
+"""The benchmark's multi-rank logic on CPU: two gloo ranks, each with its own chunk (weak
+scaling, no collective on the data path); the job time is the slowest rank's."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = [3.0, 5.0][rank]
+        ms = bench.max_over_ranks(local_ms, torch.device("cpu"))
+        dist.barrier()
+        out[rank] = ms
+        # every rank ran its own chunk: the whole-job value counts both
+        out[2 + rank] = bench.weak_scaling_value(10 ** 12, world, ms)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_max_and_count_all_work():
+    world = 2
+    out = mp.get_context("spawn").Array("d", 4)
+    mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world,
+                       start_method="spawn", join=True)
+    assert list(out[:2]) == [5.0, 5.0]
+    assert out[2] == out[3] == pytest.approx(2 * 1e12 / 5e-3 / 1e12)
+
+
+def test_single_process_is_identity():
+    assert bench.max_over_ranks(7.5, torch.device("cpu")) == 7.5
+    assert bench.weak_scaling_value(2 * 10 ** 12, 1, 1000.0) == pytest.approx(2.0)
+
+
+def test_tail_split_rule():
+    import lf_workloads as W
+    assert bench.tail_split(W.p480_shape())          # 456 tiles = 3 x 148 + 12
+    assert not bench.tail_split(W.large_shape())     # 1560 tiles = 10 x 148 + 80
