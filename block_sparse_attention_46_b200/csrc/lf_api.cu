@@ -117,12 +117,11 @@ int launch_select_frames(const Dims& D, const float* q_blk, const float* k_frm,
                          int32_t* frame_idx, float* frame_score, cudaStream_t st) {
   const size_t smem = ((size_t)D.F * (D.d + 4) + (size_t)lf::kSelWarps * D.d) * sizeof(float);
   if (smem > kMaxSmem) return LF_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(lf::select_frames_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = D.d == 128 ? lf::select_frames_kernel<128> : lf::select_frames_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return LF_ERR_CUDA;
   dim3 grid(lf::cdiv(D.nqb, lf::kSelWarps), D.H);
-  lf::select_frames_kernel<<<grid, lf::kSelWarps * 32, smem, st>>>(q_blk, k_frm, frame_idx,
-                                                                   frame_score, D);
+  kern<<<grid, lf::kSelWarps * 32, smem, st>>>(q_blk, k_frm, frame_idx, frame_score, D);
   return cuda_status(cudaGetLastError());
 }
 
@@ -132,10 +131,10 @@ int launch_select_blocks(const Dims& D, const float* q_blk, const float* k_blk,
   const size_t smem = ((size_t)D.nbpf * (D.d + 4) + (size_t)lf::kSelBatch * D.d) * sizeof(float) +
                       (size_t)D.nqb * (1 + D.kf) * sizeof(int);
   if (smem > kMaxSmem) return LF_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(lf::select_blocks_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = D.d == 128 ? lf::select_blocks_kernel<128> : lf::select_blocks_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return LF_ERR_CUDA;
-  lf::select_blocks_kernel<<<dim3(D.F, D.H), lf::kSelWarps * 32, smem, st>>>(
+  kern<<<dim3(D.F, D.H, lf::kSelSplit), lf::kSelWarps * 32, smem, st>>>(
       q_blk, k_blk, frame_idx, block_idx, block_score, D);
   return cuda_status(cudaGetLastError());
 }
@@ -223,7 +222,7 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   const int n_sm = sm_count();
   if (n_sm <= 0) return LF_ERR_CUDA;
   const AttnWs w = carve_attn(D, workspace, n_sm);
-  lf::plan_kernel<<<dim3(lf::tile_count(D), D.H), 32, 0, st>>>(
+  lf::plan_kernel<<<dim3(lf::cdiv(lf::tile_count(D), lf::kPlanWarps), D.H), lf::kPlanWarps * 32, 0, st>>>(
       D.F > 0 ? block_idx : nullptr, w.plan, w.plan_cnt, D);
   lf::schedule_kernel<<<1, 1024, 0, st>>>(w.plan_cnt, w.order, D);
   int rc = cuda_status(cudaGetLastError());

@@ -61,12 +61,18 @@ __device__ __forceinline__ int lower_bound_s(const int32_t* a, int n, int v) {
   return lo;
 }
 
-__global__ void __launch_bounds__(32)
+constexpr int kPlanWarps = 4;
+
+__global__ void __launch_bounds__(kPlanWarps * 32)
 plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
             int32_t* __restrict__ plan_cnt, const Dims D) {
-  __shared__ int32_t sa[LF_MAX_SELECTED], sb[LF_MAX_SELECTED];
-  const int t = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
+  __shared__ int32_t s_ab[kPlanWarps][2][LF_MAX_SELECTED];
   const int ntiles = tile_count(D);
+  const int t = blockIdx.x * kPlanWarps + (threadIdx.x >> 5), h = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  if (t >= ntiles) return;
+  int32_t* sa = s_ab[threadIdx.x >> 5][0];
+  int32_t* sb = s_ab[threadIdx.x >> 5][1];
   uint32_t* out = plan + ((size_t)h * ntiles + t) * plan_stride(D);
   const int nsink = D.S * D.nbpf;
   for (int e = lane; e < nsink; e += 32) out[e] = plan_pack(e / D.nbpf, e % D.nbpf, 3u);

@@ -103,15 +103,15 @@ __global__ void pool_frames_kernel(const float* __restrict__ k_blk, float* __res
   const float invT = 1.0f / (float)D.T;
   for (int c = threadIdx.x; c < D.d; c += blockDim.x) {
     float s = 0.f;
-    int b = 0;
-    for (; b + 8 <= D.nbpf; b += 8) {          // eight loads in flight, summed in block order
-      float v[8];
+    for (int b0 = 0; b0 < D.nbpf; b0 += 32) {  // 32 loads in flight, summed in block order
+      float v[32];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = src[(size_t)(b + u) * D.d + c];
+      for (int u = 0; u < 32; ++u)
+        v[u] = b0 + u < D.nbpf ? src[(size_t)(b0 + u) * D.d + c] : 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) s += (float)block_len(D, b + u) * v[u];
+      for (int u = 0; u < 32; ++u)
+        if (b0 + u < D.nbpf) s += (float)block_len(D, b0 + u) * v[u];
     }
-    for (; b < D.nbpf; ++b) s += (float)block_len(D, b) * src[(size_t)b * D.d + c];
     k_frm[((size_t)h * D.F + f) * D.d + c] = s * invT;
   }
 }
@@ -180,9 +180,11 @@ __device__ __forceinline__ void warp_write_ascending(uint32_t taken, int n, int3
 }
 
 // q . k over d channels in a fixed order (four interleaved partial sums, then combined).
-__device__ __forceinline__ float dot_fixed(const float* q, const float* k, int d) {
+template <int HD>
+__device__ __forceinline__ float dot_fixed(const float* q, const float* k) {
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  for (int c = 0; c < d; c += 4) {
+#pragma unroll
+  for (int c = 0; c < HD; c += 4) {
     const float4 x = *reinterpret_cast<const float4*>(q + c);
     const float4 y = *reinterpret_cast<const float4*>(k + c);
     a0 = fmaf(x.x, y.x, a0); a1 = fmaf(x.y, y.y, a1); a2 = fmaf(x.z, y.z, a2); a3 = fmaf(x.w, y.w, a3);
@@ -197,6 +199,7 @@ __device__ __forceinline__ float dot_fixed(const float* q, const float* k, int d
 // ---------------------------------------------------------------------------------
 constexpr int kSelWarps = 8;
 
+template <int HD>
 __global__ void __launch_bounds__(kSelWarps * 32)
 select_frames_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_frm,
                      int32_t* __restrict__ frame_idx, float* __restrict__ frame_score,
@@ -227,7 +230,7 @@ select_frames_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
     const int f = lane + 32 * j;
     float s = -INFINITY;
     if (f < D.F) {
-      s = dot_fixed(qv, sk + (size_t)f * pitch, D.d);
+      s = dot_fixed<HD>(qv, sk + (size_t)f * pitch);
       if (frame_score) frame_score[((size_t)h * D.nqb + qb) * D.F + f] = s;
     }
     sc[j] = s;
@@ -245,7 +248,9 @@ select_frames_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
 // block_idx[h, qb] — ascending overall because the frame list is ascending.
 // ---------------------------------------------------------------------------------
 constexpr int kSelBatch = 32;
+constexpr int kSelSplit = 4;      // CTAs per (frame, head): query blocks split in strides
 
+template <int HD>
 __global__ void __launch_bounds__(kSelWarps * 32)
 select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_blk,
                      const int32_t* __restrict__ frame_idx, int32_t* __restrict__ block_idx,
@@ -267,8 +272,9 @@ select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
   for (int i = threadIdx.x; i < D.nqb * D.kf; i += blockDim.x)
     s_fl[i] = frame_idx[(size_t)h * D.nqb * D.kf + i];
   __syncthreads();
-  // which query blocks chose frame f, and at which rank (lists validated on the way)
-  for (int qb = threadIdx.x; qb < D.nqb; qb += blockDim.x) {
+  // which query blocks (of this CTA's stride) chose frame f, and at which rank (lists
+  // validated on the way)
+  for (int qb = blockIdx.z + threadIdx.x * kSelSplit; qb < D.nqb; qb += blockDim.x * kSelSplit) {
     const int* fl = s_fl + (size_t)qb * D.kf;
     int rank = -1;
     bool bad = false;
@@ -280,7 +286,7 @@ select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
       if (v == f) rank = j;
     }
     if (bad) {
-      if (f == 0) record_status(LF_ERR_BAD_INDEX);
+      if (f == 0 && blockIdx.z == 0) record_status(LF_ERR_BAD_INDEX);
     } else if (rank >= 0) {
       s_list[atomicAdd(&s_n, 1)] = (qb << 10) | rank;
     }
@@ -306,7 +312,7 @@ select_blocks_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
         const int b = lane + 32 * j;
         float sres = -INFINITY;
         if (b < D.nbpf) {
-          sres = dot_fixed(qv, sk + (size_t)b * pitch, D.d);
+          sres = dot_fixed<HD>(qv, sk + (size_t)b * pitch);
           if (block_score)
             block_score[(((size_t)h * D.nqb + qb) * D.kf + rank) * D.nbpf + b] = sres;
         }
