@@ -3,9 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lf|reference] [--config 480p]
 
 One step = one pass of the whole path over one synthetic chunk: (a) token compression,
-(b) frame top-k, (c) block top-k, (d) block-sparse attention, each through its C-ABI
-entry point (lf_compress, lf_select_frames, lf_select_blocks, lf_block_sparse_attn) on
-inputs already resident in HBM.  The L2 cache is flushed (a 256 MB write) before every
+(b) frame top-k and (c) block top-k through lf_select_chunk, then (d) block-sparse
+attention through lf_block_sparse_attn, on inputs already resident in HBM.  The L2 cache is flushed (a 256 MB write) before every
 timed step, outside the step's event pair.  Reported: effective TFLOP/s = executed
 attention FLOPs (4*d per valid query-key pair) / step time; ms per chunk; roofline of the
 dominant kernel (attention, bf16 tensor cores) and of the selection (HBM); the e2e
@@ -226,11 +225,8 @@ def run_lf(args, rank, world, local_rank):
     sh = ci.shape
     nbpf, nqb, kf, kb = lf.derived(sh)
     t = {k: getattr(ci, k).to(dev) for k in ("q", "k_cur", "v_cur", "k_cache", "v_cache")}
-    q_blk = torch.empty(sh.H, nqb, sh.d, device=dev)
-    k_blk = torch.empty(sh.H, max(sh.n_hist, 1), nbpf, sh.d, device=dev)
-    k_frm = torch.empty(sh.H, max(sh.n_hist, 1), sh.d, device=dev)
-    fidx = torch.empty(sh.H, nqb, max(kf, 1), dtype=torch.int32, device=dev)
     bidx = torch.empty(sh.H, nqb, max(kf * kb, 1), dtype=torch.int32, device=dev)
+    sws = torch.empty(lf.lf_select_workspace_size(sh), dtype=torch.uint8, device=dev)
     out = torch.empty_like(t["q"])
     lse = torch.empty(sh.H, t["q"].shape[0], device=dev)
     ws = torch.empty(max(lf.lf_attn_workspace_size(sh), 256), dtype=torch.uint8, device=dev)
@@ -239,9 +235,8 @@ def run_lf(args, rank, world, local_rank):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
     def sel_stage():
-        lf.lf_compress(sh, t["q"], t["k_cache"], ci.hist_slots, q_blk, k_blk, k_frm)
-        lf.lf_select_frames(sh, q_blk, k_frm, fidx)
-        lf.lf_select_blocks(sh, q_blk, k_blk, fidx, bidx)
+        if sh.n_hist > 0:
+            lf.lf_select_chunk(sh, t["q"], t["k_cache"], ci.hist_slots, bidx, sws)
 
     def att_stage():
         lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
@@ -279,8 +274,8 @@ def run_lf(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     flops = executed_flops(sh, bidx.cpu().numpy())
-    # pool_blocks, pool_frames, select_frames, select_blocks | plan, schedule, attn (+ merge)
-    launches_per_step = (4 if sh.n_hist > 0 else 0) + 3 + (1 if tail_split(sh) else 0)
+    # pool_blocks, select_fused | plan, schedule, attn (+ merge)
+    launches_per_step = (2 if sh.n_hist > 0 else 0) + 3 + (1 if tail_split(sh) else 0)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -359,11 +354,12 @@ def run_lf(args, rank, world, local_rank):
                    "selection_share": sel_mean / (sel_mean + att_mean)},
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": att_tflops / pk["bf16_tflops"],
-                     "traffic": None, "kernel": "attn_kernel (+ plan_kernel) = stage (d)",
+                     "traffic": None,
+                     "kernel": "stage (d): plan + schedule + attn_kernel + merge (lf_block_sparse_attn)",
                      "peak_source": f"{src} bf16_tflops (burst)"},
         "roofline_selection": {"bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": sel_gbs / pk["hbm_gbs"],
-                               "kernels": "pool_blocks + pool_frames + select_frames + select_blocks",
+                               "kernels": "pool_blocks + select_fused (lf_select_chunk)",
                                "peak_source": f"{src} hbm_gbs"},
         "e2e": {"value": weak_scaling_value(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -18,6 +18,7 @@ __all__ = [
     "LfError", "LfShape", "load", "make_shape", "lf_compress", "lf_select_frames",
     "lf_select_blocks", "lf_block_sparse_attn", "lf_forward_chunk",
     "lf_attn_workspace_size", "lf_forward_workspace_size", "lf_device_status",
+    "lf_select_chunk", "lf_select_workspace_size",
     "lf_status_string", "lf_abi_version", "derived", "LIB_PATH",
 ]
 
@@ -54,6 +55,8 @@ _SIGS = {
     "lf_block_sparse_attn": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P, _P,
                                             _P, _P, _SZ, _P]),
     "lf_forward_workspace_size": (_SZ, [_SHP]),
+    "lf_select_workspace_size": (_SZ, [_SHP]),
+    "lf_select_chunk": (ctypes.c_int, [_SHP, _P, _P, _I32P, _P, _P, _SZ, _P]),
     "lf_forward_chunk": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P, _SZ, _P,
                                         _P, _P, _P]),
     "lf_device_status": (ctypes.c_int, [ctypes.c_int]),
@@ -153,6 +156,22 @@ def lf_select_blocks(shape, q_blk, k_blk, frame_idx, block_idx, block_score=None
     _check(load().lf_select_blocks(ctypes.byref(sh), _ptr(q_blk), _ptr(k_blk), _ptr(frame_idx),
                                    _ptr(block_idx), _ptr(block_score), _stream(stream)),
            "lf_select_blocks")
+
+
+def lf_select_workspace_size(shape) -> int:
+    sh = make_shape(shape)
+    return int(load().lf_select_workspace_size(ctypes.byref(sh)))
+
+
+def lf_select_chunk(shape, q, k_cache, hist_slots, block_idx, workspace=None, stream=None):
+    sh = make_shape(shape)
+    hs, _keep = _slots(hist_slots)
+    if workspace is None:
+        workspace = torch.empty(max(lf_select_workspace_size(shape), 256), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().lf_select_chunk(ctypes.byref(sh), _ptr(q), _ptr(k_cache), hs, _ptr(block_idx),
+                                  _ptr(workspace), workspace.numel(), _stream(stream)),
+           "lf_select_chunk")
 
 
 def lf_attn_workspace_size(shape) -> int:

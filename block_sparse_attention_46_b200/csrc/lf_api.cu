@@ -10,6 +10,7 @@
 #include "lf_common.cuh"
 #include "lf_select.cuh"
 #include "lf_attn.cuh"
+#include "lf_fused.cuh"
 
 using lf::Dims;
 
@@ -109,7 +110,8 @@ int launch_compress(const Dims& D, const void* q, const void* k_cache, const int
   const int vecs = D.H * D.d / 8;
   dim3 grid(units, lf::cdiv(vecs, lf::kPoolThreads));
   lf::pool_blocks_kernel<<<grid, lf::kPoolThreads, 0, st>>>(a, D);
-  if (D.F > 0) lf::pool_frames_kernel<<<dim3(D.F, D.H), D.d, 0, st>>>(k_blk, k_frm, D);
+  if (D.F > 0 && k_frm != nullptr)
+    lf::pool_frames_kernel<<<dim3(D.F, D.H), D.d, 0, st>>>(k_blk, k_frm, D);
   return cuda_status(cudaGetLastError());
 }
 
@@ -218,12 +220,14 @@ int launch_attn_t(const Dims& D, lf::AttnParams& p, int grid, cudaStream_t st) {
 int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_cur,
                 const void* k_cache, const void* v_cache, const int32_t* hist_slots,
                 const int32_t* sink_slots, const int32_t* block_idx, void* out, float* lse,
-                void* workspace, cudaStream_t st) {
+                void* workspace, cudaStream_t st, bool plans_ready = false) {
   const int n_sm = sm_count();
   if (n_sm <= 0) return LF_ERR_CUDA;
   const AttnWs w = carve_attn(D, workspace, n_sm);
-  lf::plan_kernel<<<dim3(lf::cdiv(lf::tile_count(D), lf::kPlanWarps), D.H), lf::kPlanWarps * 32, 0, st>>>(
-      D.F > 0 ? block_idx : nullptr, w.plan, w.plan_cnt, D);
+  // key plans (unless the fused selection already wrote them), then the launch order
+  if (!plans_ready)
+    lf::plan_kernel<<<dim3(lf::cdiv(lf::tile_count(D), lf::kPlanWarps), D.H), lf::kPlanWarps * 32, 0, st>>>(
+        D.F > 0 ? block_idx : nullptr, w.plan, w.plan_cnt, D);
   lf::schedule_kernel<<<1, 1024, 0, st>>>(w.plan_cnt, w.order, D);
   int rc = cuda_status(cudaGetLastError());
   if (rc != LF_OK) return rc;
@@ -285,6 +289,36 @@ FwdWs carve(const Dims& D, void* base) {
   w.attn = take(attn_ws_bytes(D));
   w.bytes = off;
   return w;
+}
+
+// Stages (a)-(c) into `bidx`: pooling, then the fused selection (which also writes the
+// attention key plans into the workspace) when the shape allows it, else the separate
+// frame-pooling, frame-selection and block-selection kernels.
+int run_select(const Dims& D, const void* q, const void* k_cache, const int32_t* hist_slots,
+               const FwdWs& w, int32_t* bidx, cudaStream_t stream, bool* plans_ready) {
+  int rc;
+  *plans_ready = false;
+  if (lf::fused_select_ok(D) && lf::fused_select_smem(D) <= kMaxSmem) {
+    if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, nullptr, stream)) != LF_OK)
+      return rc;
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return LF_ERR_CUDA;
+    const AttnWs aw = carve_attn(D, w.attn, n_sm);
+    const size_t smem = lf::fused_select_smem(D);
+    auto kern = D.d == 128 ? lf::select_fused_kernel<128> : lf::select_fused_kernel<64>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return LF_ERR_CUDA;
+    kern<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), 256, smem, stream>>>(
+        w.q_blk, w.k_blk, bidx, aw.plan, aw.plan_cnt, D);
+    if ((rc = cuda_status(cudaGetLastError())) != LF_OK) return rc;
+    *plans_ready = true;
+    return LF_OK;
+  }
+  if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, w.k_frm, stream)) != LF_OK)
+    return rc;
+  if ((rc = launch_select_frames(D, w.q_blk, w.k_frm, w.frame_idx, nullptr, stream)) != LF_OK)
+    return rc;
+  return launch_select_blocks(D, w.q_blk, w.k_blk, w.frame_idx, bidx, nullptr, stream);
 }
 
 }  // namespace
@@ -410,16 +444,31 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
     return LF_ERR_WORKSPACE;
   const FwdWs w = carve(D, workspace);
   int32_t* bidx = block_idx_out ? block_idx_out : w.block_idx;
-  if (D.F > 0) {
-    if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, w.k_frm, stream)) != LF_OK)
-      return rc;
-    if ((rc = launch_select_frames(D, w.q_blk, w.k_frm, w.frame_idx, nullptr, stream)) != LF_OK)
-      return rc;
-    if ((rc = launch_select_blocks(D, w.q_blk, w.k_blk, w.frame_idx, bidx, nullptr, stream)) != LF_OK)
-      return rc;
-  }
+  bool plans_ready = false;
+  if (D.F > 0 && (rc = run_select(D, q, k_cache, hist_slots, w, bidx, stream, &plans_ready)) != LF_OK)
+    return rc;
   return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, bidx, out,
-                     lse, w.attn, stream);
+                     lse, w.attn, stream, plans_ready);
+}
+
+size_t lf_select_workspace_size(const lf_shape* shape) { return lf_forward_workspace_size(shape); }
+
+int lf_select_chunk(const lf_shape* shape, const void* q, const void* k_cache,
+                    const int32_t* hist_slots, int32_t* block_idx, void* workspace,
+                    size_t workspace_bytes, cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (D.F < 1) return LF_ERR_INVALID_ARG;
+  if (q == nullptr || k_cache == nullptr || block_idx == nullptr || !aligned(q, 16) ||
+      !aligned(k_cache, 16) || !aligned(block_idx, 4))
+    return LF_ERR_INVALID_ARG;
+  if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
+  const FwdWs need = carve(D, nullptr);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need.bytes)
+    return LF_ERR_WORKSPACE;
+  bool plans_ready = false;
+  return run_select(D, q, k_cache, hist_slots, carve(D, workspace), block_idx, stream, &plans_ready);
 }
 
 int lf_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {

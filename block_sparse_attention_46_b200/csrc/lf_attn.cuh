@@ -61,6 +61,47 @@ __device__ __forceinline__ int lower_bound_s(const int32_t* a, int n, int v) {
   return lo;
 }
 
+// One warp writes a tile's key plan from its query blocks' ascending block lists A and
+// B (shared memory, already validated; nB = 0 when the tile has one query block): sink
+// blocks first, then the sorted union.  Returns the entry count.
+__device__ __forceinline__ int warp_write_plan(const int32_t* sa, int nA, const int32_t* sb,
+                                               int nB, uint32_t* out, const Dims& D) {
+  const int lane = threadIdx.x & 31;
+  const int nsink = D.S * D.nbpf;
+  for (int e = lane; e < nsink; e += 32) out[e] = plan_pack(e / D.nbpf, e % D.nbpf, 3u);
+  const uint32_t lt = (1u << lane) - 1u;
+  int carry = 0;
+  for (int i0 = 0; i0 < nA; i0 += 32) {
+    const int i = i0 + lane;
+    const bool valid = i < nA;
+    const int a = valid ? sa[i] : 0x7fffffff;
+    const int cb = lower_bound_s(sb, nB, a);
+    const bool inB = valid && cb < nB && sb[cb] == a;
+    const uint32_t bal = __ballot_sync(0xffffffffu, inB);
+    if (valid) {
+      const int pos = i + cb - (carry + __popc(bal & lt));
+      out[nsink + pos] = plan_pack(D.S + a / D.nbpf, a % D.nbpf, inB ? 3u : 1u);
+    }
+    carry += __popc(bal);
+  }
+  const int ncommon = carry;
+  carry = 0;
+  for (int j0 = 0; j0 < nB; j0 += 32) {
+    const int j = j0 + lane;
+    const bool valid = j < nB;
+    const int b = valid ? sb[j] : 0x7fffffff;
+    const int ca = lower_bound_s(sa, nA, b);
+    const bool inA = valid && ca < nA && sa[ca] == b;
+    const uint32_t bal = __ballot_sync(0xffffffffu, inA);
+    if (valid && !inA) {
+      const int pos = j + ca - (carry + __popc(bal & lt));
+      out[nsink + pos] = plan_pack(D.S + b / D.nbpf, b % D.nbpf, 2u);
+    }
+    carry += __popc(bal);
+  }
+  return nsink + nA + nB - ncommon;
+}
+
 constexpr int kPlanWarps = 4;
 
 __global__ void __launch_bounds__(kPlanWarps * 32)
@@ -74,13 +115,12 @@ plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
   int32_t* sa = s_ab[threadIdx.x >> 5][0];
   int32_t* sb = s_ab[threadIdx.x >> 5][1];
   uint32_t* out = plan + ((size_t)h * ntiles + t) * plan_stride(D);
-  const int nsink = D.S * D.nbpf;
-  for (int e = lane; e < nsink; e += 32) out[e] = plan_pack(e / D.nbpf, e % D.nbpf, 3u);
-  int cnt = nsink;
+  int nA = 0, nB = 0;
   if (D.F > 0 && D.nsel > 0 && block_idx != nullptr) {
     const int qa = D.B == 64 ? 2 * t : t;
     const int qbB = (D.B == 64 && 2 * t + 1 < D.nqb) ? 2 * t + 1 : -1;
-    const int nA = D.nsel, nB = qbB >= 0 ? D.nsel : 0;
+    nA = D.nsel;
+    nB = qbB >= 0 ? D.nsel : 0;
     const int32_t* A = block_idx + ((size_t)h * D.nqb + qa) * D.nsel;
     const int32_t* B = qbB >= 0 ? block_idx + ((size_t)h * D.nqb + qbB) * D.nsel : nullptr;
     const int lim = D.F * D.nbpf;
@@ -92,42 +132,12 @@ plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
       bad |= sa[i] < 0 || sa[i] >= lim || (i > 0 && sa[i - 1] >= sa[i]);
     for (int i = lane; i < nB; i += 32)
       bad |= sb[i] < 0 || sb[i] >= lim || (i > 0 && sb[i - 1] >= sb[i]);
-    if (__any_sync(0xffffffffu, bad)) {
+    if (__any_sync(0xffffffffu, bad)) {       // the selected lists are dropped
       if (lane == 0) record_status(LF_ERR_BAD_INDEX);
-    } else {
-      const uint32_t lt = (1u << lane) - 1u;
-      int carry = 0;
-      for (int i0 = 0; i0 < nA; i0 += 32) {
-        const int i = i0 + lane;
-        const bool valid = i < nA;
-        const int a = valid ? sa[i] : 0x7fffffff;
-        const int cb = lower_bound_s(sb, nB, a);
-        const bool inB = valid && cb < nB && sb[cb] == a;
-        const uint32_t bal = __ballot_sync(0xffffffffu, inB);
-        if (valid) {
-          const int pos = i + cb - (carry + __popc(bal & lt));
-          out[nsink + pos] = plan_pack(D.S + a / D.nbpf, a % D.nbpf, inB ? 3u : 1u);
-        }
-        carry += __popc(bal);
-      }
-      const int ncommon = carry;
-      carry = 0;
-      for (int j0 = 0; j0 < nB; j0 += 32) {
-        const int j = j0 + lane;
-        const bool valid = j < nB;
-        const int b = valid ? sb[j] : 0x7fffffff;
-        const int ca = lower_bound_s(sa, nA, b);
-        const bool inA = valid && ca < nA && sa[ca] == b;
-        const uint32_t bal = __ballot_sync(0xffffffffu, inA);
-        if (valid && !inA) {
-          const int pos = j + ca - (carry + __popc(bal & lt));
-          out[nsink + pos] = plan_pack(D.S + b / D.nbpf, b % D.nbpf, 2u);
-        }
-        carry += __popc(bal);
-      }
-      cnt = nsink + nA + nB - ncommon;
+      nA = nB = 0;
     }
   }
+  const int cnt = warp_write_plan(sa, nA, sb, nB, out, D);
   if (lane == 0) plan_cnt[(size_t)h * ntiles + t] = cnt;
 }
 

@@ -114,6 +114,17 @@ int lf_select_blocks(const lf_shape* shape, const float* q_blk, const float* k_b
                      const int32_t* frame_idx, int32_t* block_idx, float* block_score,
                      cudaStream_t stream);
 
+/* (a)+(b)+(c) in one call [LF-gist 2.2; LF-yly 三]: pooling, frame top-k and block top-k.
+ * block_idx (device, [H, n_qb, kf*kb]) receives the selected global block ids, ascending
+ * per (h, qb), exactly as lf_compress + lf_select_frames + lf_select_blocks define them
+ * (frame scores use the identity q_blk . k_frm = sum_b len_b (q_blk . k_blk[b]) / T).
+ * workspace: at least lf_select_workspace_size(shape) bytes, 256-byte aligned.
+ * Requires n_hist >= 1. */
+size_t lf_select_workspace_size(const lf_shape* shape);
+int lf_select_chunk(const lf_shape* shape, const void* q, const void* k_cache,
+                    const int32_t* hist_slots, int32_t* block_idx, void* workspace,
+                    size_t workspace_bytes, cudaStream_t stream);
+
 /* Workspace bytes lf_block_sparse_attn needs for this shape (its per-tile key plans). */
 size_t lf_attn_workspace_size(const lf_shape* shape);
 

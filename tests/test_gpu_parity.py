@@ -111,6 +111,23 @@ def test_small_all_stages(gpu_lib, name):
     assert gpu_lib.lf_device_status() == 0
 
 
+@pytest.mark.parametrize("name", [n for n in SMALL if n not in ("no_history", "sinks_only")])
+def test_select_chunk_matches_oracle(gpu_lib, name):
+    """(a)+(b)+(c) in one call against the oracle's two-stage selection."""
+    ci = SMALL[name]()
+    sh = ci.shape
+    t = G.to_dev(ci)
+    nbpf, nqb, kf, kb = gpu_lib.derived(sh)
+    bidx = torch.full((sh.H, nqb, kf * kb), -7, dtype=torch.int32, device="cuda")
+    gpu_lib.lf_select_chunk(sh, t["q"], t["k_cache"], ci.hist_slots, bidx)
+    torch.cuda.synchronize()
+    qb, kb_, kf_, fidx, sf, oidx, sb = _oracle_selection(ci)
+    gaps = np.minimum(G.frame_gaps(sf, kf), G.block_gaps(sb, kb))
+    bad, near, n = G.compare_indices(bidx.cpu().numpy(), oidx, gaps)
+    assert bad == 0, f"{name}: {bad}/{n} lists differ outside near ties"
+    assert gpu_lib.lf_device_status() == 0
+
+
 def _full_size_check(ci, samples):
     """The benchmark's call on a full-size workload; all indices against the oracle,
     output on sampled query blocks (oracle attention given the GPU's own mask)."""
