@@ -270,7 +270,7 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
 
 // forward workspace carve-up
 struct FwdWs {
-  float *q_blk, *k_blk, *k_frm;
+  float *q_blk, *k_blk, *k_frm, *scores;
   int32_t *frame_idx, *block_idx;
   void* attn;
   size_t bytes;
@@ -284,6 +284,7 @@ FwdWs carve(const Dims& D, void* base) {
   w.q_blk = reinterpret_cast<float*>(take((size_t)D.H * D.nqb * D.d * 4));
   w.k_blk = reinterpret_cast<float*>(take((size_t)D.H * D.F * D.nbpf * D.d * 4));
   w.k_frm = reinterpret_cast<float*>(take((size_t)D.H * D.F * D.d * 4));
+  w.scores = reinterpret_cast<float*>(take((size_t)D.H * D.nqb * D.F * D.nbpf * 4));
   w.frame_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.kf * 4));
   w.block_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.nsel * 4));
   w.attn = take(attn_ws_bytes(D));
@@ -304,12 +305,15 @@ int run_select(const Dims& D, const void* q, const void* k_cache, const int32_t*
     const int n_sm = sm_count();
     if (n_sm <= 0) return LF_ERR_CUDA;
     const AttnWs aw = carve_attn(D, w.attn, n_sm);
+    const dim3 sgrid(lf::cdiv(D.F * D.nbpf, lf::kScoreRows), D.H, lf::cdiv(D.nqb, lf::kScoreQb));
+    if (D.d == 128) lf::block_scores_kernel<128><<<sgrid, 256, 0, stream>>>(w.q_blk, w.k_blk, w.scores, D);
+    else lf::block_scores_kernel<64><<<sgrid, 256, 0, stream>>>(w.q_blk, w.k_blk, w.scores, D);
     const size_t smem = lf::fused_select_smem(D);
-    auto kern = D.d == 128 ? lf::select_fused_kernel<128> : lf::select_fused_kernel<64>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(lf::select_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
       return LF_ERR_CUDA;
-    kern<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), 256, smem, stream>>>(
-        w.q_blk, w.k_blk, bidx, aw.plan, aw.plan_cnt, D);
+    lf::select_pick_kernel<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), 256, smem, stream>>>(
+        w.scores, bidx, aw.plan, aw.plan_cnt, D);
     if ((rc = cuda_status(cudaGetLastError())) != LF_OK) return rc;
     *plans_ready = true;
     return LF_OK;

@@ -1,13 +1,11 @@
-// lf_fused.cuh — stages (b) and (c) fused, with the attention key plans, for the
-// one-call path (lf_forward_chunk).
-//
-// Per (head, group of kFuseQb query blocks): the scores of every history block against
-// the group's pooled queries (a small GEMM, q_blk[8 x d] . k_blk[F*n_bpf x d]^T, fixed
-// summation order), the frame scores from them by linearity (a frame's pooled key is the
-// length-weighted mean of its block keys, so its score is the length-weighted mean of
-// the block scores), the top-k_f frames, the top-k_b blocks in each chosen frame, and the
-// key plans of the group's query tiles.  [LF-gist 2.2] two-stage mask selection;
-// [LF-yly 三] inner-product similarity.
+// lf_fused.cuh — stages (b) and (c) for the one-call paths (lf_select_chunk,
+// lf_forward_chunk): every history block's score against every pooled query block (a
+// small GEMM, q_blk . k_blk^T, fixed summation order), then per group of query blocks the
+// frame scores from them by linearity (a frame's pooled key is the length-weighted mean of
+// its block keys, so its score is the length-weighted mean of the block scores), the
+// top-k_f frames, the top-k_b blocks in each chosen frame, and the key plans of the
+// group's query tiles.  [LF-gist 2.2] two-stage mask selection; [LF-yly 三] inner-product
+// similarity.
 #pragma once
 #include "lf_select.cuh"
 #include "lf_attn.cuh"
@@ -24,66 +22,78 @@ __host__ __device__ inline bool fused_select_ok(const Dims& D) {
 }
 
 __host__ __device__ inline size_t fused_select_smem(const Dims& D) {
-  return (size_t)kFuseQb * D.d * 4 + (size_t)kFuseQb * D.F * D.nbpf * 4 +
-         (size_t)kFuseQb * D.nsel * 4 + (size_t)kFuseQb * D.kf * 4;
+  return (size_t)kFuseQb * D.F * D.nbpf * 4 + (size_t)kFuseQb * D.nsel * 4 +
+         (size_t)kFuseQb * D.kf * 4;
 }
+
+// Scores of every history block against every pooled query block of head h:
+// s[h, qb, r] = q_blk[h, qb] . k_blk[h, r], r = f * n_bpf + b.  CTA = (64 rows, head,
+// 16 query blocks); rows and queries are staged in shared memory with coalesced loads;
+// thread (row, quarter) computes four query blocks against one row, each score one
+// fixed-order sum over the channels.
+constexpr int kScoreRows = 64, kScoreQb = 16;
 
 template <int HD>
 __global__ void __launch_bounds__(256)
-select_fused_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_blk,
-                    int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
-                    int32_t* __restrict__ plan_cnt, const Dims D) {
-  extern __shared__ float4 sm4[];
-  float* sq = reinterpret_cast<float*>(sm4);                       // [kFuseQb][HD]
+block_scores_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_blk,
+                    float* __restrict__ scores, const Dims D) {
+  __shared__ float4 sk4[kScoreRows * (HD / 4 + 1)];
+  __shared__ float4 sq4[kScoreQb * (HD / 4)];
   const int NB = D.F * D.nbpf;
-  float* sc = sq + kFuseQb * HD;                                    // [kFuseQb][NB]
+  const int r0 = blockIdx.x * kScoreRows, h = blockIdx.y, q0 = blockIdx.z * kScoreQb;
+  const int pitch = HD / 4 + 1;                       // float4 pitch, padded
+  for (int i = threadIdx.x; i < kScoreRows * (HD / 4); i += blockDim.x) {
+    const int r = i / (HD / 4), c4 = i % (HD / 4);
+    sk4[r * pitch + c4] = r0 + r < NB
+        ? __ldg(reinterpret_cast<const float4*>(k_blk + ((size_t)h * NB + r0 + r) * HD) + c4)
+        : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int i = threadIdx.x; i < kScoreQb * (HD / 4); i += blockDim.x) {
+    const int g = i / (HD / 4), c4 = i % (HD / 4);
+    sq4[i] = q0 + g < D.nqb
+        ? __ldg(reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + q0 + g) * HD) + c4)
+        : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  const int r = threadIdx.x % kScoreRows, gq = threadIdx.x / kScoreRows;   // 4 quarters
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+  for (int c4 = 0; c4 < HD / 4; ++c4) {
+    const float4 k = sk4[r * pitch + c4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 q = sq4[(gq * 4 + u) * (HD / 4) + c4];
+      acc[u] = fmaf(q.x, k.x, acc[u]); acc[u] = fmaf(q.y, k.y, acc[u]);
+      acc[u] = fmaf(q.z, k.z, acc[u]); acc[u] = fmaf(q.w, k.w, acc[u]);
+    }
+  }
+  if (r0 + r < NB)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int qb = q0 + gq * 4 + u;
+      if (qb < D.nqb) scores[((size_t)h * D.nqb + qb) * NB + r0 + r] = acc[u];
+    }
+}
+
+// Per (head, group of kFuseQb query blocks): frame scores by linearity from the block
+// scores, frame top-k, block top-k in each chosen frame, block_idx, and the key plans of
+// the group's query tiles.
+__global__ void __launch_bounds__(256)
+select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block_idx,
+                   uint32_t* __restrict__ plan, int32_t* __restrict__ plan_cnt, const Dims D) {
+  extern __shared__ float4 sm4[];
+  const int NB = D.F * D.nbpf;
+  float* sc = reinterpret_cast<float*>(sm4);                        // [kFuseQb][NB]
   int32_t* sl = reinterpret_cast<int32_t*>(sc + (size_t)kFuseQb * NB);   // [kFuseQb][nsel]
   int32_t* sf = sl + kFuseQb * D.nsel;                              // [kFuseQb][kf]
   const int h = blockIdx.y, qb0 = blockIdx.x * kFuseQb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  for (int i = threadIdx.x; i < kFuseQb * (HD / 4); i += blockDim.x) {
-    const int g = i / (HD / 4), c4 = i % (HD / 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (qb0 + g < D.nqb)
-      v = reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + qb0 + g) * HD)[c4];
-    reinterpret_cast<float4*>(sq + g * HD)[c4] = v;
+  for (int i = threadIdx.x; i < kFuseQb * NB; i += blockDim.x) {
+    const int g = i / NB, r = i % NB;
+    sc[i] = qb0 + g < D.nqb ? scores[((size_t)h * D.nqb + qb0 + g) * NB + r] : 0.f;
   }
   __syncthreads();
 
-  // block scores: thread t takes rows t, t + 256, ... of k_blk[h] (two at a time); each
-  // score is one fixed-order sum over the channels
-  const float* kh = k_blk + (size_t)h * NB * HD;
-  for (int r0 = threadIdx.x; r0 < NB; r0 += 2 * blockDim.x) {
-    const int r1 = r0 + blockDim.x;
-    const bool has1 = r1 < NB;
-    float acc0[kFuseQb], acc1[kFuseQb];
-#pragma unroll
-    for (int g = 0; g < kFuseQb; ++g) acc0[g] = acc1[g] = 0.f;
-    const float4* k0 = reinterpret_cast<const float4*>(kh + (size_t)r0 * HD);
-    const float4* k1 = reinterpret_cast<const float4*>(kh + (size_t)(has1 ? r1 : r0) * HD);
-#pragma unroll 4
-    for (int c4 = 0; c4 < HD / 4; ++c4) {
-      const float4 a = __ldg(k0 + c4);
-      const float4 b = __ldg(k1 + c4);
-#pragma unroll
-      for (int g = 0; g < kFuseQb; ++g) {
-        const float4 q = reinterpret_cast<const float4*>(sq + g * HD)[c4];
-        acc0[g] = fmaf(q.x, a.x, acc0[g]); acc0[g] = fmaf(q.y, a.y, acc0[g]);
-        acc0[g] = fmaf(q.z, a.z, acc0[g]); acc0[g] = fmaf(q.w, a.w, acc0[g]);
-        acc1[g] = fmaf(q.x, b.x, acc1[g]); acc1[g] = fmaf(q.y, b.y, acc1[g]);
-        acc1[g] = fmaf(q.z, b.z, acc1[g]); acc1[g] = fmaf(q.w, b.w, acc1[g]);
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < kFuseQb; ++g) {
-      sc[(size_t)g * NB + r0] = acc0[g];
-      if (has1) sc[(size_t)g * NB + r1] = acc1[g];
-    }
-  }
-  __syncthreads();
-
-  // per query block (warp g): frame scores, frame top-k, block top-k in chosen frames
   const float invT = 1.0f / (float)D.T;
   for (int g = warp; g < kFuseQb; g += blockDim.x / 32) {
     const int qb = qb0 + g;

@@ -29,7 +29,7 @@ struct PoolArgs {
 };
 
 constexpr int kPoolThreads = 64;
-constexpr int kPoolUnroll = 8;
+constexpr int kPoolUnroll = 16;
 
 __global__ void __launch_bounds__(kPoolThreads)
 pool_blocks_kernel(const __grid_constant__ PoolArgs a, const Dims D) {
