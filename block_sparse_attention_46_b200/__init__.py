@@ -18,7 +18,8 @@ __all__ = [
     "LfError", "LfShape", "load", "make_shape", "lf_compress", "lf_select_frames",
     "lf_select_blocks", "lf_block_sparse_attn", "lf_forward_chunk",
     "lf_attn_workspace_size", "lf_forward_workspace_size", "lf_device_status",
-    "lf_select_chunk", "lf_select_workspace_size",
+    "lf_select_chunk", "lf_select_workspace_size", "lf_block_sparse_attn_noalloc",
+    "lf_noalloc_scratch_bytes",
     "lf_status_string", "lf_abi_version", "derived", "LIB_PATH",
 ]
 
@@ -63,6 +64,9 @@ _SIGS = {
     "lf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "lf_abi_version": (ctypes.c_int, []),
     "lf_debug_exp2_poly": (ctypes.c_int, [_P, _P, ctypes.c_int, _P]),
+    "lf_noalloc_scratch_bytes": (_SZ, []),
+    "lf_block_sparse_attn_noalloc": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P,
+                                                    _P, _P, _P]),
 }
 
 
@@ -196,6 +200,23 @@ def lf_block_sparse_attn(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, s
         ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_cache), _ptr(v_cache), hs, ss,
         _ptr(block_idx), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)), "lf_block_sparse_attn")
+
+
+def lf_noalloc_scratch_bytes() -> int:
+    return int(load().lf_noalloc_scratch_bytes())
+
+
+def lf_block_sparse_attn_noalloc(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots,
+                                 sink_slots, block_idx, out, lse=None, stream=None):
+    """lf_block_sparse_attn without a workspace argument, for callers that cannot
+    allocate device memory: the library's fixed scratch array is used instead (calls
+    that overlap on the GPU must not share a device)."""
+    sh = make_shape(shape)
+    hs, _k1 = _slots(hist_slots)
+    ss, _k2 = _slots(sink_slots)
+    _check(load().lf_block_sparse_attn_noalloc(
+        ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_cache), _ptr(v_cache), hs, ss,
+        _ptr(block_idx), _ptr(out), _ptr(lse), _stream(stream)), "lf_block_sparse_attn_noalloc")
 
 
 def lf_forward_chunk(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,

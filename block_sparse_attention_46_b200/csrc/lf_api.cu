@@ -325,6 +325,33 @@ int run_select(const Dims& D, const void* q, const void* k_cache, const int32_t*
   return launch_select_blocks(D, w.q_blk, w.k_blk, w.frame_idx, bidx, nullptr, stream);
 }
 
+// ---------------------------------------------------------------- fixed scratch
+// Scratch for lf_block_sparse_attn_noalloc: a fixed-size array in device global memory
+// that every device loading this library holds until the process exits.  Host code
+// must not use the symbol itself as a device address; the device address is obtained
+// once per device with cudaGetSymbolAddress (with that device current) and cached.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;       // 16 MiB
+static __device__ __align__(256) uint8_t g_lf_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the fixed scratch on the current device (set up on first use).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_lf_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return LF_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return LF_OK;
+}
+
 }  // namespace
 
 // ===================================================================== C ABI
@@ -418,6 +445,25 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
     return LF_ERR_WORKSPACE;
   return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, block_idx,
                      out, lse, workspace, stream);
+}
+
+size_t lf_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+int lf_block_sparse_attn_noalloc(const lf_shape* shape, const void* q, const void* k_cur,
+                                 const void* v_cur, const void* k_cache, const void* v_cache,
+                                 const int32_t* hist_slots, const int32_t* sink_slots,
+                                 const int32_t* block_idx, void* out, float* lse,
+                                 cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  const size_t need = attn_ws_bytes(D);
+  if (need == 0) return LF_ERR_CUDA;
+  if (need > kNoAllocScratchBytes) return LF_ERR_WORKSPACE;   // shape needs more scratch
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch)) != LF_OK) return rc;
+  return lf_block_sparse_attn(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
+                              block_idx, out, lse, scratch, kNoAllocScratchBytes, stream);
 }
 
 size_t lf_forward_workspace_size(const lf_shape* shape) {

@@ -145,6 +145,33 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
                          const int32_t* block_idx, void* out, float* lse,
                          void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* lf_block_sparse_attn for callers that cannot allocate device memory.
+ *
+ * No counterpart in the paper: this is a packaging variant of (d).  Some callers cannot
+ * provide the workspace lf_block_sparse_attn asks for: code embedded in a host runtime
+ * that exposes no allocator or scratch hook to it, or a latency-critical loop that allows
+ * no device allocation after start-up (cudaMalloc may synchronise the device).  This
+ * entry point takes the same arguments minus the workspace and uses instead a fixed
+ * scratch array in device global memory that lives in the library: at most
+ * lf_noalloc_scratch_bytes() bytes (16 MiB), reserved on every device that loads the
+ * library until the process exits.  It allocates nothing and calls no allocating routine.
+ *
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *    with that device current) and caches it; make that first call before any stream
+ *    capture on the device.
+ *  - All calls on a device share the one array, which keeps the last call's contents
+ *    (nothing in it needs to start at zero).  Calls whose work may overlap on the GPU —
+ *    on different streams, or from different host threads — race on it; serialise them.
+ *  - A shape whose workspace (lf_attn_workspace_size) exceeds the array returns
+ *    LF_ERR_WORKSPACE without launching anything.
+ * Results are those of lf_block_sparse_attn. */
+size_t lf_noalloc_scratch_bytes(void);
+int lf_block_sparse_attn_noalloc(const lf_shape* shape, const void* q, const void* k_cur,
+                                 const void* v_cur, const void* k_cache, const void* v_cache,
+                                 const int32_t* hist_slots, const int32_t* sink_slots,
+                                 const int32_t* block_idx, void* out, float* lse,
+                                 cudaStream_t stream);
+
 /* Workspace bytes lf_forward_chunk needs: pooled tensors, index lists and key plans. */
 size_t lf_forward_workspace_size(const lf_shape* shape);
 
