@@ -239,7 +239,7 @@ def run_lf(args, rank, world, local_rank):
         # write 256 MB (> 126 MB of L2), then read it back: L2 ends up holding clean lines
         # of the flush buffer, so no dirty write-back is charged to the timed kernels
         flush.zero_()
-        torch.sum(flush.view(torch.int64), out=flush_sink)
+        torch.sum(flush.view(torch.int64), dim=0, out=flush_sink)
     stream = torch.cuda.current_stream()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
