@@ -108,7 +108,7 @@ int launch_compress(const Dims& D, const void* q, const void* k_cache, const int
   for (int f = 0; f < D.F; ++f) a.hist_slots[f] = hist_slots[f];
   const int units = D.nqb + D.F * D.nbpf;
   const int vecs = D.H * D.d / 8;
-  dim3 grid(units, lf::cdiv(vecs, lf::kPoolThreads));
+  dim3 grid(units, lf::cdiv(vecs, lf::kPoolCols));
   lf::pool_blocks_kernel<<<grid, lf::kPoolThreads, 0, st>>>(a, D);
   if (D.F > 0 && k_frm != nullptr)
     lf::pool_frames_kernel<<<dim3(D.F, D.H), D.d, 0, st>>>(k_blk, k_frm, D);

@@ -125,8 +125,8 @@ plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
     const int32_t* B = qbB >= 0 ? block_idx + ((size_t)h * D.nqb + qbB) * D.nsel : nullptr;
     const int lim = D.F * D.nbpf;
     bool bad = false;
-    for (int i = lane; i < nA; i += 32) sa[i] = A[i];
-    for (int i = lane; i < nB; i += 32) sb[i] = B[i];
+    stage_words(sa, A, nA, lane, 32);
+    if (nB > 0) stage_words(sb, B, nB, lane, 32);
     __syncwarp();
     for (int i = lane; i < nA; i += 32)
       bad |= sa[i] < 0 || sa[i] >= lim || (i > 0 && sa[i - 1] >= sa[i]);
@@ -380,10 +380,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     LF_TR_CTA(1, globaltimer_ns());
     LF_TR_CTA(3, n_iter);
   }
-  if (warp == 3) {
-    const uint32_t* src = P.plan + (size_t)tile * plan_stride(D);
-    for (int i = lane; i < cnt; i += 32) s_plan[i] = src[i];
-  }
+  if (warp == 3) stage_words(s_plan, P.plan + (size_t)tile * plan_stride(D), cnt, lane, 32);
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&P.tm_q); prefetch_tmap(&P.tm_kc); prefetch_tmap(&P.tm_kh);
     prefetch_tmap(&P.tm_vc); prefetch_tmap(&P.tm_vh);

@@ -66,6 +66,23 @@ __device__ __forceinline__ uint32_t smid() {
   return r;
 }
 
+// Block-cooperative copy of n 32-bit words from global to shared memory with up to eight
+// loads in flight per thread (a plain loop would wait for each load before the next).
+template <typename T>
+__device__ __forceinline__ void stage_words(T* __restrict__ dst, const T* __restrict__ src,
+                                            int n, int tid, int nthreads) {
+  static_assert(sizeof(T) == 4, "32-bit words");
+  int i = tid;
+  for (; i + 7 * nthreads < n; i += 8 * nthreads) {
+    T v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = src[i + u * nthreads];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) dst[i + u * nthreads] = v[u];
+  }
+  for (; i < n; i += nthreads) dst[i] = src[i];
+}
+
 // ------------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -34,7 +34,7 @@ __host__ __device__ inline size_t fused_select_smem(const Dims& D) {
 constexpr int kScoreRows = 64, kScoreQb = 16;
 
 template <int HD>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256)   // staging assumes exactly 256 threads
 block_scores_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_blk,
                     float* __restrict__ scores, const Dims D) {
   __shared__ float4 sk4[kScoreRows * (HD / 4 + 1)];
@@ -42,17 +42,35 @@ block_scores_kernel(const float* __restrict__ q_blk, const float* __restrict__ k
   const int NB = D.F * D.nbpf;
   const int r0 = blockIdx.x * kScoreRows, h = blockIdx.y, q0 = blockIdx.z * kScoreQb;
   const int pitch = HD / 4 + 1;                       // float4 pitch, padded
-  for (int i = threadIdx.x; i < kScoreRows * (HD / 4); i += blockDim.x) {
-    const int r = i / (HD / 4), c4 = i % (HD / 4);
-    sk4[r * pitch + c4] = r0 + r < NB
-        ? __ldg(reinterpret_cast<const float4*>(k_blk + ((size_t)h * NB + r0 + r) * HD) + c4)
-        : make_float4(0.f, 0.f, 0.f, 0.f);
+  {
+    // kScoreRows * HD / 4 float4 = 2048 (d = 128): eight loads in flight per thread
+    constexpr int n4 = kScoreRows * (HD / 4);
+    float4 v[n4 / 256];
+#pragma unroll
+    for (int u = 0; u < n4 / 256; ++u) {
+      const int i = threadIdx.x + u * 256, r = i / (HD / 4), c4 = i % (HD / 4);
+      v[u] = r0 + r < NB
+          ? __ldg(reinterpret_cast<const float4*>(k_blk + ((size_t)h * NB + r0 + r) * HD) + c4)
+          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < n4 / 256; ++u) {
+      const int i = threadIdx.x + u * 256, r = i / (HD / 4), c4 = i % (HD / 4);
+      sk4[r * pitch + c4] = v[u];
+    }
   }
-  for (int i = threadIdx.x; i < kScoreQb * (HD / 4); i += blockDim.x) {
-    const int g = i / (HD / 4), c4 = i % (HD / 4);
-    sq4[i] = q0 + g < D.nqb
-        ? __ldg(reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + q0 + g) * HD) + c4)
-        : make_float4(0.f, 0.f, 0.f, 0.f);
+  {
+    constexpr int n4 = kScoreQb * (HD / 4);
+    float4 v[n4 / 256];
+#pragma unroll
+    for (int u = 0; u < n4 / 256; ++u) {
+      const int i = threadIdx.x + u * 256, g = i / (HD / 4), c4 = i % (HD / 4);
+      v[u] = q0 + g < D.nqb
+          ? __ldg(reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + q0 + g) * HD) + c4)
+          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < n4 / 256; ++u) sq4[threadIdx.x + u * 256] = v[u];
   }
   __syncthreads();
   const int r = threadIdx.x % kScoreRows, gq = threadIdx.x / kScoreRows;   // 4 quarters
@@ -88,9 +106,10 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
   int32_t* sf = sl + kFuseQb * D.nsel;                              // [kFuseQb][kf]
   const int h = blockIdx.y, qb0 = blockIdx.x * kFuseQb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kFuseQb * NB; i += blockDim.x) {
-    const int g = i / NB, r = i % NB;
-    sc[i] = qb0 + g < D.nqb ? scores[((size_t)h * D.nqb + qb0 + g) * NB + r] : 0.f;
+  {
+    // the group's rows of the score matrix are contiguous: [qb0, qb0 + kFuseQb) x NB
+    const int ng = min(kFuseQb, D.nqb - qb0);
+    stage_words(sc, scores + ((size_t)h * D.nqb + qb0) * NB, ng * NB, threadIdx.x, blockDim.x);
   }
   __syncthreads();
 

@@ -18,7 +18,9 @@ namespace lf {
 // (a) Pooling.  One CTA row (blockIdx.x) is one block of tokens: the first nqb rows are
 // the current chunk's query blocks, the next F*nbpf rows the history key blocks.  Each
 // thread owns 8 consecutive channels of the H*d-wide token row (one 16-byte load per
-// token), so a warp reads 512 contiguous bytes per token.  Sums are fp32, token order.
+// token), so a warp reads 512 contiguous bytes per token.  Sums are fp32 in a fixed
+// order: four consecutive runs of the block's tokens, each in token order, then the runs
+// in order.
 // ---------------------------------------------------------------------------------
 struct PoolArgs {
   const __nv_bfloat16* q;        // [ncur, H, d]
@@ -28,15 +30,21 @@ struct PoolArgs {
   int hist_slots[LF_MAX_FRAMES];
 };
 
-constexpr int kPoolThreads = 64;
+constexpr int kPoolCols = 64;       // 8-channel groups per CTA (threads per token group)
+constexpr int kPoolGroups = 4;      // token groups per CTA: a block's tokens split in 4 runs
+constexpr int kPoolThreads = kPoolCols * kPoolGroups;
 constexpr int kPoolUnroll = 16;
 
-__global__ void __launch_bounds__(kPoolThreads)
+// Thread (token group g, column group c): sums its run of the block's tokens in token order
+// (16-byte loads, up to 16 in flight); the four runs are then added in run order.
+__global__ void __launch_bounds__(kPoolThreads, 2)
 pool_blocks_kernel(const __grid_constant__ PoolArgs a, const Dims D) {
+  __shared__ float part[kPoolGroups][kPoolCols][8];
   const int unit = blockIdx.x;
   const int HD = D.H * D.d;
-  const int vec = blockIdx.y * kPoolThreads + threadIdx.x;   // 8-channel group
-  if (vec * 8 >= HD) return;
+  const int col = threadIdx.x % kPoolCols, g = threadIdx.x / kPoolCols;
+  const int vec = blockIdx.y * kPoolCols + col;               // 8-channel group
+  const bool active = vec * 8 < HD;
 
   const __nv_bfloat16* base;
   int ntok;
@@ -55,43 +63,46 @@ pool_blocks_kernel(const __grid_constant__ PoolArgs a, const Dims D) {
     base = a.k_cache + ((size_t)slot * D.T + (size_t)b * D.B) * HD;
     dst = a.k_blk + (((size_t)h * D.F + f) * D.nbpf + b) * D.d + c0;
   }
+  const int run = (ntok + kPoolGroups - 1) / kPoolGroups;
+  const int t0 = g * run, t1 = min(ntok, t0 + run);
   const uint4* src = reinterpret_cast<const uint4*>(base) + vec;
   const size_t stride = HD / 8;     // uint4 per token row
 
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-
-  int t = 0;
-  for (; t + kPoolUnroll <= ntok; t += kPoolUnroll) {
-    uint4 v[kPoolUnroll];
+  if (active) {
+    for (int t = t0; t < t1; t += kPoolUnroll) {
+      uint4 v[kPoolUnroll];
 #pragma unroll
-    for (int u = 0; u < kPoolUnroll; ++u) v[u] = __ldg(src + (size_t)(t + u) * stride);
+      for (int u = 0; u < kPoolUnroll; ++u)
+        if (t + u < t1) v[u] = __ldg(src + (size_t)(t + u) * stride);
 #pragma unroll
-    for (int u = 0; u < kPoolUnroll; ++u) {
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+      for (int u = 0; u < kPoolUnroll; ++u) {
+        if (t + u < t1) {
+          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float2 f2 = __bfloat1622float2(p[i]);
-        acc[2 * i] += f2.x;
-        acc[2 * i + 1] += f2.y;
+          for (int i = 0; i < 4; ++i) {
+            const float2 f2 = __bfloat1622float2(p[i]);
+            acc[2 * i] += f2.x;
+            acc[2 * i + 1] += f2.y;
+          }
+        }
       }
     }
   }
-  for (; t < ntok; ++t) {
-    uint4 v = __ldg(src + (size_t)t * stride);
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 f2 = __bfloat1622float2(p[i]);
-      acc[2 * i] += f2.x;
-      acc[2 * i + 1] += f2.y;
-    }
-  }
+  for (int i = 0; i < 8; ++i) part[g][col][i] = acc[i];
+  __syncthreads();
+  if (g != 0 || !active) return;
+  float s[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    s[i] = ((part[0][col][i] + part[1][col][i]) + part[2][col][i]) + part[3][col][i];
   const float inv = 1.0f / (float)ntok;
   float4* o = reinterpret_cast<float4*>(dst);
-  o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  o[0] = make_float4(s[0] * inv, s[1] * inv, s[2] * inv, s[3] * inv);
+  o[1] = make_float4(s[4] * inv, s[5] * inv, s[6] * inv, s[7] * inv);
 }
 
 // Frame pooling from the block means: k_frm = sum_b len_b * k_blk[b] / T (the frame mean
