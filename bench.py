@@ -72,6 +72,51 @@ def tail_split(shape, n_sm=148) -> bool:
     return r != 0 and 2 * r <= n_sm
 
 
+def selection_launches(shape) -> int:
+    """Kernels one lf_select_chunk call launches (mirrors the library's rule): pooling,
+    block scores and pick when the fused path applies, else pooling, frame pooling, frame
+    selection and block selection."""
+    if shape.n_hist <= 0:
+        return 0
+    nbpf = -(-shape.T // shape.block)
+    kf, kb = min(shape.k_f, shape.n_hist), min(shape.k_b, nbpf)
+    fused = (shape.n_hist * nbpf <= 2048 and kf * kb <= 256 and shape.n_hist <= 256
+             and nbpf <= 256)
+    return 3 if fused else 4
+
+
+def attn_sources_sha256() -> str:
+    """Digest of the attention kernel's sources (the DRAM traffic figure taken from an ncu
+    capture is reported only while the kernel is unchanged)."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_46_b200", "csrc")
+    for name in ("lf_attn.cuh", "lf_common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary of this workload,
+    or None if there is none or the kernel's sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != attn_sources_sha256():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def max_over_ranks(x: float, device) -> float:
     """The largest value of x over all ranks (the job's time is its slowest rank's)."""
     import torch
@@ -283,8 +328,8 @@ def run_lf(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     flops = executed_flops(sh, bidx.cpu().numpy())
-    # pool_blocks, select_fused | plan, schedule, attn (+ merge)
-    launches_per_step = (2 if sh.n_hist > 0 else 0) + 3 + (1 if tail_split(sh) else 0)
+    # selection kernels | plan, schedule, attn (+ merge)
+    launches_per_step = selection_launches(sh) + 3 + (1 if tail_split(sh) else 0)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -364,12 +409,12 @@ def run_lf(args, rank, world, local_rank):
                    "selection_share": sel_mean / (sel_mean + att_mean)},
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": att_tflops / pk["bf16_tflops"],
-                     "traffic": None,
+                     "traffic": profiled_traffic(args.config),
                      "kernel": "stage (d): plan + schedule + attn_kernel + merge (lf_block_sparse_attn)",
                      "peak_source": f"{src} bf16_tflops (burst)"},
         "roofline_selection": {"bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": sel_gbs / pk["hbm_gbs"],
-                               "kernels": "pool_blocks + select_fused (lf_select_chunk)",
+                               "kernels": "pool_blocks + block_scores + select_pick (lf_select_chunk)",
                                "peak_source": f"{src} hbm_gbs"},
         "e2e": {"value": weak_scaling_value(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
