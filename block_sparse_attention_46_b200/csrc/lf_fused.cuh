@@ -12,7 +12,13 @@
 
 namespace lf {
 
-constexpr int kFuseQb = 8;                 // query blocks per CTA (even: whole tile pairs)
+#ifndef LF_FUSE_QB
+#define LF_FUSE_QB 8
+#endif
+#ifndef LF_SCORE_QB
+#define LF_SCORE_QB 16
+#endif
+constexpr int kFuseQb = LF_FUSE_QB;        // query blocks per CTA (even: whole tile pairs)
 constexpr int kFuseMaxBlocks = 2048;       // F * n_bpf handled by the fused path
 constexpr int kFuseMaxSel = 256;           // k_f * k_b handled by the fused path
 
@@ -28,10 +34,12 @@ __host__ __device__ inline size_t fused_select_smem(const Dims& D) {
 
 // Scores of every history block against every pooled query block of head h:
 // s[h, qb, r] = q_blk[h, qb] . k_blk[h, r], r = f * n_bpf + b.  CTA = (64 rows, head,
-// 16 query blocks); rows and queries are staged in shared memory with coalesced loads;
-// thread (row, quarter) computes four query blocks against one row, each score one
-// fixed-order sum over the channels.
-constexpr int kScoreRows = 64, kScoreQb = 16;
+// kScoreQb query blocks); rows and queries are staged in shared memory with coalesced
+// loads; thread (row, quarter) computes kScoreQb / 4 query blocks against one row, each
+// score one fixed-order sum over the channels.
+constexpr int kScoreRows = 64, kScoreQb = LF_SCORE_QB;
+constexpr int kScoreQpt = kScoreQb * kScoreRows / 256;    // query blocks per thread
+static_assert(kScoreQpt >= 1 && kScoreQpt * 256 == kScoreQb * kScoreRows, "score tiling");
 
 template <int HD>
 __global__ void __launch_bounds__(256)   // staging assumes exactly 256 threads
@@ -59,36 +67,31 @@ block_scores_kernel(const float* __restrict__ q_blk, const float* __restrict__ k
       sk4[r * pitch + c4] = v[u];
     }
   }
-  {
-    constexpr int n4 = kScoreQb * (HD / 4);
-    float4 v[n4 / 256];
-#pragma unroll
-    for (int u = 0; u < n4 / 256; ++u) {
-      const int i = threadIdx.x + u * 256, g = i / (HD / 4), c4 = i % (HD / 4);
-      v[u] = q0 + g < D.nqb
-          ? __ldg(reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + q0 + g) * HD) + c4)
-          : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < n4 / 256; ++u) sq4[threadIdx.x + u * 256] = v[u];
+  for (int i = threadIdx.x; i < kScoreQb * (HD / 4); i += 256) {
+    const int g = i / (HD / 4), c4 = i % (HD / 4);
+    sq4[i] = q0 + g < D.nqb
+        ? __ldg(reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + q0 + g) * HD) + c4)
+        : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
   const int r = threadIdx.x % kScoreRows, gq = threadIdx.x / kScoreRows;   // 4 quarters
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc[kScoreQpt];
+#pragma unroll
+  for (int u = 0; u < kScoreQpt; ++u) acc[u] = 0.f;
 #pragma unroll 8
   for (int c4 = 0; c4 < HD / 4; ++c4) {
     const float4 k = sk4[r * pitch + c4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 q = sq4[(gq * 4 + u) * (HD / 4) + c4];
+    for (int u = 0; u < kScoreQpt; ++u) {
+      const float4 q = sq4[(gq * kScoreQpt + u) * (HD / 4) + c4];
       acc[u] = fmaf(q.x, k.x, acc[u]); acc[u] = fmaf(q.y, k.y, acc[u]);
       acc[u] = fmaf(q.z, k.z, acc[u]); acc[u] = fmaf(q.w, k.w, acc[u]);
     }
   }
   if (r0 + r < NB)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int qb = q0 + gq * 4 + u;
+    for (int u = 0; u < kScoreQpt; ++u) {
+      const int qb = q0 + gq * kScoreQpt + u;
       if (qb < D.nqb) scores[((size_t)h * D.nqb + qb) * NB + r0 + r] = acc[u];
     }
 }
