@@ -356,6 +356,52 @@ def run_lf(args, rank, world, local_rank):
     ms_step = total_ms / args.steps
     value = weak_scaling_value(flops, world, ms_step)
 
+    # incremental compression: history block means kept per cache slot; per step the frames
+    # that enter the cache (three slots re-pooled here, their keys unchanged, so the
+    # selection is the same) are pooled and the selection reads the pooled-key cache
+    inc = None
+    if sh.n_hist > 0:
+        k_pool = torch.empty(lf.lf_pooled_cache_bytes(sh) // 4, dtype=torch.float32, device=dev)
+        lf.lf_pool_frames(sh, t["k_cache"], sorted(set(ci.hist_slots)), k_pool)
+        new_slots = list(ci.hist_slots[:sh.n_cur_frames])
+        bidx_c = torch.empty_like(bidx)
+
+        def sel_cached():
+            lf.lf_pool_frames(sh, t["k_cache"], new_slots, k_pool)
+            lf.lf_select_chunk_cached(sh, t["q"], k_pool, ci.hist_slots, bidx_c, sws)
+        for _ in range(3):
+            sel_cached()
+        torch.cuda.synchronize()
+        g_selc = torch.cuda.CUDAGraph()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g_selc, stream=cap):
+                sel_cached()
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+        n_inc = max(3, min(args.steps, 200))
+        selc_ms, attc_ms = [], []
+        for _ in range(n_inc):
+            flush_l2()
+            ev[0].record(stream)
+            g_selc.replay()
+            ev[1].record(stream)
+            g_att.replay()
+            ev[2].record(stream)
+            ev[2].synchronize()
+            selc_ms.append(ev[0].elapsed_time(ev[1]))
+            attc_ms.append(ev[1].elapsed_time(ev[2]))
+        same = bool(torch.equal(bidx_c, bidx))
+        inc_bytes = 2 * sh.H * sh.d * sh.T * (2 * sh.n_cur_frames)      # Q + the new frames' K
+        selc_mean = max_over_ranks(statistics.mean(selc_ms), dev)
+        inc = {"ms_selection_abc": selc_mean,
+               "ms_per_step": selc_mean + max_over_ranks(statistics.mean(attc_ms), dev),
+               "selection_mb_per_chunk": inc_bytes / 1e6,
+               "selection_gbs": inc_bytes / (selc_mean * 1e-3) / 1e9,
+               "indices_equal_full_recompute": same,
+               "api": "lf_pool_frames (the chunk's frames entering the cache) + "
+                      "lf_select_chunk_cached, then lf_block_sparse_attn"}
+
     # e2e through lf_forward_chunk with host buffers: every step copies its chunk's Q, K, V
     # from pinned host memory, runs the call, and copies the output back.  Two chunks are
     # in flight: uploads, compute and downloads run on three streams (separate copy
@@ -439,6 +485,7 @@ def run_lf(args, rank, world, local_rank):
                 "api": "lf_forward_chunk per step, two chunks in flight (uploads, compute and "
                        "downloads on three streams)",
                 "output_equals_device_path": e2e_same},
+        "incremental_compression": inc,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }

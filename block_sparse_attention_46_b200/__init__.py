@@ -19,7 +19,8 @@ __all__ = [
     "lf_select_blocks", "lf_block_sparse_attn", "lf_forward_chunk",
     "lf_attn_workspace_size", "lf_forward_workspace_size", "lf_device_status",
     "lf_select_chunk", "lf_select_workspace_size", "lf_block_sparse_attn_noalloc",
-    "lf_noalloc_scratch_bytes",
+    "lf_noalloc_scratch_bytes", "lf_pooled_cache_bytes", "lf_pool_frames",
+    "lf_select_chunk_cached",
     "lf_status_string", "lf_abi_version", "derived", "LIB_PATH",
 ]
 
@@ -65,6 +66,9 @@ _SIGS = {
     "lf_abi_version": (ctypes.c_int, []),
     "lf_debug_exp2_poly": (ctypes.c_int, [_P, _P, ctypes.c_int, _P]),
     "lf_noalloc_scratch_bytes": (_SZ, []),
+    "lf_pooled_cache_bytes": (_SZ, [_SHP]),
+    "lf_pool_frames": (ctypes.c_int, [_SHP, _P, _I32P, ctypes.c_int32, _P, _P]),
+    "lf_select_chunk_cached": (ctypes.c_int, [_SHP, _P, _P, _I32P, _P, _P, _SZ, _P]),
     "lf_block_sparse_attn_noalloc": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P,
                                                     _P, _P, _P]),
 }
@@ -176,6 +180,31 @@ def lf_select_chunk(shape, q, k_cache, hist_slots, block_idx, workspace=None, st
     _check(load().lf_select_chunk(ctypes.byref(sh), _ptr(q), _ptr(k_cache), hs, _ptr(block_idx),
                                   _ptr(workspace), workspace.numel(), _stream(stream)),
            "lf_select_chunk")
+
+
+def lf_pooled_cache_bytes(shape) -> int:
+    sh = make_shape(shape)
+    return int(load().lf_pooled_cache_bytes(ctypes.byref(sh)))
+
+
+def lf_pool_frames(shape, k_cache, slots, k_pool, stream=None):
+    """Block means of the keys of cache slots `slots` into the pooled-key cache k_pool
+    (fp32 [n_slots, H, n_bpf, d])."""
+    sh = make_shape(shape)
+    sl, _keep = _slots(slots)
+    _check(load().lf_pool_frames(ctypes.byref(sh), _ptr(k_cache), sl, len(slots), _ptr(k_pool),
+                                 _stream(stream)), "lf_pool_frames")
+
+
+def lf_select_chunk_cached(shape, q, k_pool, hist_slots, block_idx, workspace=None, stream=None):
+    sh = make_shape(shape)
+    hs, _keep = _slots(hist_slots)
+    if workspace is None:
+        workspace = torch.empty(max(lf_select_workspace_size(shape), 256), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().lf_select_chunk_cached(ctypes.byref(sh), _ptr(q), _ptr(k_pool), hs,
+                                         _ptr(block_idx), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)), "lf_select_chunk_cached")
 
 
 def lf_attn_workspace_size(shape) -> int:

@@ -105,6 +105,7 @@ int launch_compress(const Dims& D, const void* q, const void* k_cache, const int
   a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   a.q_blk = q_blk;
   a.k_blk = k_blk;
+  a.k_pool = nullptr;
   for (int f = 0; f < D.F; ++f) a.hist_slots[f] = hist_slots[f];
   const int units = D.nqb + D.F * D.nbpf;
   const int vecs = D.H * D.d / 8;
@@ -112,6 +113,23 @@ int launch_compress(const Dims& D, const void* q, const void* k_cache, const int
   lf::pool_blocks_kernel<<<grid, lf::kPoolThreads, 0, st>>>(a, D);
   if (D.F > 0 && k_frm != nullptr)
     lf::pool_frames_kernel<<<dim3(D.F, D.H), D.d, 0, st>>>(k_blk, k_frm, D);
+  return cuda_status(cudaGetLastError());
+}
+
+// Block means of the keys of cache slots `slots[0..n)` into the pooled-key cache
+// k_pool [n_slots, H, nbpf, d] (the pooling kernel over history units only).
+int launch_pool_frames(const Dims& D, const void* k_cache, const int32_t* slots, int n,
+                       float* k_pool, cudaStream_t st) {
+  if (n == 0) return LF_OK;
+  Dims Dp = D;
+  Dp.nqb = 0;
+  Dp.F = n;
+  lf::PoolArgs a{};
+  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  a.k_pool = k_pool;
+  for (int f = 0; f < n; ++f) a.hist_slots[f] = slots[f];
+  dim3 grid(n * D.nbpf, lf::cdiv(D.H * D.d / 8, lf::kPoolCols));
+  lf::pool_blocks_kernel<<<grid, lf::kPoolThreads, 0, st>>>(a, Dp);
   return cuda_status(cudaGetLastError());
 }
 
@@ -292,6 +310,30 @@ FwdWs carve(const Dims& D, void* base) {
   return w;
 }
 
+// Block scores (from the per-call pooled keys w.k_blk, or from the pooled-key cache k_pool
+// through hist_slots) and the pick kernel (frame and block top-k, key plans).
+int launch_scores_pick(const Dims& D, const FwdWs& w, const float* k_pool,
+                       const int32_t* hist_slots, const AttnWs& aw, int32_t* bidx,
+                       cudaStream_t stream) {
+  lf::ScoreArgs sa{};
+  sa.q_blk = w.q_blk;
+  sa.k_blk = w.k_blk;
+  sa.k_pool = k_pool;
+  sa.scores = w.scores;
+  if (k_pool != nullptr)
+    for (int f = 0; f < D.F; ++f) sa.slots[f] = hist_slots[f];
+  const dim3 sgrid(lf::cdiv(D.F * D.nbpf, lf::kScoreRows), D.H, lf::cdiv(D.nqb, lf::kScoreQb));
+  if (D.d == 128) lf::block_scores_kernel<128><<<sgrid, 256, 0, stream>>>(sa, D);
+  else lf::block_scores_kernel<64><<<sgrid, 256, 0, stream>>>(sa, D);
+  const size_t smem = lf::fused_select_smem(D);
+  if (cudaFuncSetAttribute(lf::select_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return LF_ERR_CUDA;
+  lf::select_pick_kernel<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), 256, smem, stream>>>(
+      w.scores, bidx, aw.plan, aw.plan_cnt, D);
+  return cuda_status(cudaGetLastError());
+}
+
 // Stages (a)-(c) into `bidx`: pooling, then the fused selection (which also writes the
 // attention key plans into the workspace) when the shape allows it, else the separate
 // frame-pooling, frame-selection and block-selection kernels.
@@ -305,16 +347,7 @@ int run_select(const Dims& D, const void* q, const void* k_cache, const int32_t*
     const int n_sm = sm_count();
     if (n_sm <= 0) return LF_ERR_CUDA;
     const AttnWs aw = carve_attn(D, w.attn, n_sm);
-    const dim3 sgrid(lf::cdiv(D.F * D.nbpf, lf::kScoreRows), D.H, lf::cdiv(D.nqb, lf::kScoreQb));
-    if (D.d == 128) lf::block_scores_kernel<128><<<sgrid, 256, 0, stream>>>(w.q_blk, w.k_blk, w.scores, D);
-    else lf::block_scores_kernel<64><<<sgrid, 256, 0, stream>>>(w.q_blk, w.k_blk, w.scores, D);
-    const size_t smem = lf::fused_select_smem(D);
-    if (cudaFuncSetAttribute(lf::select_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return LF_ERR_CUDA;
-    lf::select_pick_kernel<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), 256, smem, stream>>>(
-        w.scores, bidx, aw.plan, aw.plan_cnt, D);
-    if ((rc = cuda_status(cudaGetLastError())) != LF_OK) return rc;
+    if ((rc = launch_scores_pick(D, w, nullptr, hist_slots, aw, bidx, stream)) != LF_OK) return rc;
     *plans_ready = true;
     return LF_OK;
   }
@@ -519,6 +552,51 @@ int lf_select_chunk(const lf_shape* shape, const void* q, const void* k_cache,
     return LF_ERR_WORKSPACE;
   bool plans_ready = false;
   return run_select(D, q, k_cache, hist_slots, carve(D, workspace), block_idx, stream, &plans_ready);
+}
+
+size_t lf_pooled_cache_bytes(const lf_shape* shape) {
+  Dims D;
+  if (make_dims(shape, &D) != LF_OK) return 0;
+  return (size_t)D.n_slots * D.H * D.nbpf * D.d * sizeof(float);
+}
+
+int lf_pool_frames(const lf_shape* shape, const void* k_cache, const int32_t* slots,
+                   int32_t n, float* k_pool, cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (n < 0 || n > LF_MAX_FRAMES) return LF_ERR_INVALID_ARG;
+  if (n == 0) return LF_OK;
+  if (k_cache == nullptr || k_pool == nullptr || !aligned(k_cache, 16) || !aligned(k_pool, 16))
+    return LF_ERR_INVALID_ARG;
+  if ((rc = check_slots(slots, n, D.n_slots)) != LF_OK) return rc;
+  return launch_pool_frames(D, k_cache, slots, n, k_pool, stream);
+}
+
+int lf_select_chunk_cached(const lf_shape* shape, const void* q, const float* k_pool,
+                           const int32_t* hist_slots, int32_t* block_idx, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (D.F < 1) return LF_ERR_INVALID_ARG;
+  if (q == nullptr || k_pool == nullptr || block_idx == nullptr || !aligned(q, 16) ||
+      !aligned(k_pool, 16) || !aligned(block_idx, 4))
+    return LF_ERR_INVALID_ARG;
+  if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
+  if (!lf::fused_select_ok(D) || lf::fused_select_smem(D) > kMaxSmem) return LF_ERR_UNSUPPORTED;
+  const FwdWs need = carve(D, nullptr);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need.bytes)
+    return LF_ERR_WORKSPACE;
+  const FwdWs w = carve(D, workspace);
+  Dims Dq = D;
+  Dq.F = 0;                                  // pool the query blocks only
+  if ((rc = launch_compress(Dq, q, nullptr, hist_slots, w.q_blk, nullptr, nullptr, stream)) != LF_OK)
+    return rc;
+  const int n_sm = sm_count();
+  if (n_sm <= 0) return LF_ERR_CUDA;
+  return launch_scores_pick(D, w, k_pool, hist_slots, carve_attn(D, w.attn, n_sm), block_idx,
+                            stream);
 }
 
 int lf_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {

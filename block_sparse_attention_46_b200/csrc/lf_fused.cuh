@@ -41,10 +41,19 @@ constexpr int kScoreRows = 64, kScoreQb = LF_SCORE_QB;
 constexpr int kScoreQpt = kScoreQb * kScoreRows / 256;    // query blocks per thread
 static_assert(kScoreQpt >= 1 && kScoreQpt * 256 == kScoreQb * kScoreRows, "score tiling");
 
+struct ScoreArgs {
+  const float* q_blk;   // [H, nqb, d]
+  const float* k_blk;   // [H, F, nbpf, d], or null when k_pool is used
+  const float* k_pool;  // [n_slots, H, nbpf, d] pooled-key cache, read through slots[]
+  float* scores;        // [H, nqb, F * nbpf]
+  int slots[LF_MAX_FRAMES];
+};
+
 template <int HD>
 __global__ void __launch_bounds__(256)   // staging assumes exactly 256 threads
-block_scores_kernel(const float* __restrict__ q_blk, const float* __restrict__ k_blk,
-                    float* __restrict__ scores, const Dims D) {
+block_scores_kernel(const __grid_constant__ ScoreArgs a, const Dims D) {
+  const float* __restrict__ q_blk = a.q_blk;
+  float* __restrict__ scores = a.scores;
   __shared__ float4 sk4[kScoreRows * (HD / 4 + 1)];
   __shared__ float4 sq4[kScoreQb * (HD / 4)];
   const int NB = D.F * D.nbpf;
@@ -57,9 +66,14 @@ block_scores_kernel(const float* __restrict__ q_blk, const float* __restrict__ k
 #pragma unroll
     for (int u = 0; u < n4 / 256; ++u) {
       const int i = threadIdx.x + u * 256, r = i / (HD / 4), c4 = i % (HD / 4);
-      v[u] = r0 + r < NB
-          ? __ldg(reinterpret_cast<const float4*>(k_blk + ((size_t)h * NB + r0 + r) * HD) + c4)
-          : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int rr = r0 + r;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (rr < NB) {
+        const float* row = a.k_pool != nullptr
+            ? a.k_pool + (((size_t)a.slots[rr / D.nbpf] * D.H + h) * D.nbpf + rr % D.nbpf) * HD
+            : a.k_blk + ((size_t)h * NB + rr) * HD;
+        v[u] = __ldg(reinterpret_cast<const float4*>(row) + c4);
+      }
     }
 #pragma unroll
     for (int u = 0; u < n4 / 256; ++u) {

@@ -27,6 +27,8 @@ struct PoolArgs {
   const __nv_bfloat16* k_cache;  // [n_slots, T, H, d]
   float* q_blk;                  // [H, nqb, d]
   float* k_blk;                  // [H, F, nbpf, d]
+  float* k_pool;                 // [n_slots, H, nbpf, d] pooled-key cache, or null: when
+                                 // set, history blocks are written to their slot's rows
   int hist_slots[LF_MAX_FRAMES];
 };
 
@@ -61,7 +63,9 @@ pool_blocks_kernel(const __grid_constant__ PoolArgs a, const Dims D) {
     const int slot = a.hist_slots[f];
     ntok = block_len(D, b);
     base = a.k_cache + ((size_t)slot * D.T + (size_t)b * D.B) * HD;
-    dst = a.k_blk + (((size_t)h * D.F + f) * D.nbpf + b) * D.d + c0;
+    dst = a.k_pool != nullptr
+        ? a.k_pool + (((size_t)slot * D.H + h) * D.nbpf + b) * D.d + c0
+        : a.k_blk + (((size_t)h * D.F + f) * D.nbpf + b) * D.d + c0;
   }
   const int run = (ntok + kPoolGroups - 1) / kPoolGroups;
   const int t0 = g * run, t1 = min(ntok, t0 + run);

@@ -125,6 +125,32 @@ int lf_select_chunk(const lf_shape* shape, const void* q, const void* k_cache,
                     const int32_t* hist_slots, int32_t* block_idx, void* workspace,
                     size_t workspace_bytes, cudaStream_t stream);
 
+/* Pooled-key cache (incremental compression).  A frame's keys do not change once it is
+ * in the KV cache [SF, rolling KV cache paragraph], so its block means [LF-gist 2.2,
+ * token compression] can be computed once, when the frame enters, instead of on every
+ * call.  The pages describe no such cache; it changes no result: the cached path
+ * selects bit-identically to lf_select_chunk.
+ *
+ * k_pool (device, caller-owned, fp32 [n_slots, H, n_bpf, d], lf_pooled_cache_bytes):
+ * row (slot, h, b) holds the mean of block b of the keys in cache slot `slot`, computed
+ * exactly as lf_compress computes k_blk.
+ *
+ * lf_pool_frames: pools the keys of the n cache slots slots[0..n) (HOST array, each in
+ * [0, n_slots)) of k_cache [n_slots, T, H, d] bf16 into their rows of k_pool; other rows
+ * are untouched.  0 <= n <= LF_MAX_FRAMES; n == 0 does nothing.
+ *
+ * lf_select_chunk_cached: lf_select_chunk with the history block means read from k_pool
+ * through hist_slots (their rows must have been written by lf_pool_frames since the
+ * slots' keys last changed); only the current chunk's queries are pooled.  Same
+ * workspace as lf_select_chunk.  Returns LF_ERR_UNSUPPORTED for shapes beyond the fused
+ * selection's limits (n_hist * n_bpf > 2048 or k_f * k_b > 256).  Requires n_hist >= 1. */
+size_t lf_pooled_cache_bytes(const lf_shape* shape);
+int lf_pool_frames(const lf_shape* shape, const void* k_cache, const int32_t* slots,
+                   int32_t n, float* k_pool, cudaStream_t stream);
+int lf_select_chunk_cached(const lf_shape* shape, const void* q, const float* k_pool,
+                           const int32_t* hist_slots, int32_t* block_idx, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
+
 /* Workspace bytes lf_block_sparse_attn needs for this shape (its per-tile key plans). */
 size_t lf_attn_workspace_size(const lf_shape* shape);
 

@@ -95,3 +95,32 @@ def test_workspace_sizes(lib):
 def test_status_strings(lib):
     assert lf.lf_status_string(0) == "ok"
     assert "timed out" in lf.lf_status_string(4)
+
+
+def _i32(vals):
+    arr = (ctypes.c_int32 * max(len(vals), 1))(*vals)
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)), arr
+
+
+def test_pooled_cache_validation(lib):
+    sh = lf.make_shape(_shape())
+    slots, _k = _i32([0, 3])
+    bad, _k2 = _i32([0, 4])                                             # slot >= n_slots
+    assert lib.lf_pool_frames(ctypes.byref(sh), FAKE, slots, 0, FAKE, None) == 0   # nothing
+    assert lib.lf_pool_frames(ctypes.byref(sh), FAKE, bad, 2, FAKE, None) == 1
+    assert lib.lf_pool_frames(ctypes.byref(sh), FAKE, slots, -1, FAKE, None) == 1
+    assert lib.lf_pool_frames(ctypes.byref(sh), FAKE, slots, 257, FAKE, None) == 1
+    assert lib.lf_pool_frames(ctypes.byref(sh), None, slots, 2, FAKE, None) == 1
+    assert lib.lf_pool_frames(ctypes.byref(sh), FAKE, slots, 2, ctypes.c_void_p((1 << 20) + 4),
+                              None) == 1                                # misaligned cache
+    hist, _k3 = _i32([0, 1, 2, 3])
+    assert lib.lf_select_chunk_cached(ctypes.byref(sh), FAKE, FAKE, hist, FAKE, None, 0,
+                                      None) == 5                        # no workspace
+    assert lib.lf_select_chunk_cached(ctypes.byref(sh), FAKE, None, hist, FAKE, FAKE, 1 << 30,
+                                      None) == 1                        # no pooled cache
+    nh = lf.make_shape(_shape(n_hist=0, n_slots=0))
+    assert lib.lf_select_chunk_cached(ctypes.byref(nh), FAKE, FAKE, hist, FAKE, FAKE, 1 << 30,
+                                      None) == 1                        # needs history
+    # the cache holds one fp32 row of d channels per (slot, head, block)
+    s480 = W.p480_shape()
+    assert lf.lf_pooled_cache_bytes(s480) == s480.n_slots * 12 * 25 * 128 * 4
