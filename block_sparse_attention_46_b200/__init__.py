@@ -20,7 +20,7 @@ __all__ = [
     "lf_attn_workspace_size", "lf_forward_workspace_size", "lf_device_status",
     "lf_select_chunk", "lf_select_workspace_size", "lf_block_sparse_attn_noalloc",
     "lf_noalloc_scratch_bytes", "lf_pooled_cache_bytes", "lf_pool_frames",
-    "lf_select_chunk_cached",
+    "lf_select_chunk_cached", "lf_cag_schedule",
     "lf_status_string", "lf_abi_version", "derived", "LIB_PATH",
 ]
 
@@ -67,6 +67,9 @@ _SIGS = {
     "lf_debug_exp2_poly": (ctypes.c_int, [_P, _P, ctypes.c_int, _P]),
     "lf_noalloc_scratch_bytes": (_SZ, []),
     "lf_pooled_cache_bytes": (_SZ, [_SHP]),
+    "lf_cag_schedule": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                                       ctypes.c_float, _I32P, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.POINTER(ctypes.c_float), _I32P, _I32P]),
     "lf_pool_frames": (ctypes.c_int, [_SHP, _P, _I32P, ctypes.c_int32, _P, _P]),
     "lf_select_chunk_cached": (ctypes.c_int, [_SHP, _P, _P, _I32P, _P, _P, _SZ, _P]),
     "lf_block_sparse_attn_noalloc": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P,
@@ -205,6 +208,27 @@ def lf_select_chunk_cached(shape, q, k_pool, hist_slots, block_idx, workspace=No
     _check(load().lf_select_chunk_cached(ctypes.byref(sh), _ptr(q), _ptr(k_pool), hs,
                                          _ptr(block_idx), _ptr(workspace), workspace.numel(),
                                          _stream(stream)), "lf_select_chunk_cached")
+
+
+def lf_cag_schedule(n_chunks, first, mean_sparsity, final_sparsity, n_hist=None, n_bpf=1,
+                    kf_max=1):
+    """Per-chunk keep ratios of the chunk-aware sparsity growth, and (if n_hist is given)
+    the (k_f, k_b) budgets.  Host only.  Returns (keep, k_f, k_b); the last two are None
+    without n_hist."""
+    keep = (ctypes.c_float * n_chunks)()
+    if n_hist is not None:
+        nh = (ctypes.c_int32 * n_chunks)(*[int(x) for x in n_hist])
+        kf = (ctypes.c_int32 * n_chunks)()
+        kb = (ctypes.c_int32 * n_chunks)()
+        args = (ctypes.cast(nh, _I32P), n_bpf, kf_max, keep, ctypes.cast(kf, _I32P),
+                ctypes.cast(kb, _I32P))
+    else:
+        args = (None, n_bpf, kf_max, keep, None, None)
+    _check(load().lf_cag_schedule(n_chunks, first, mean_sparsity, final_sparsity, *args),
+           "lf_cag_schedule")
+    if n_hist is None:
+        return list(keep), None, None
+    return list(keep), list(kf), list(kb)
 
 
 def lf_attn_workspace_size(shape) -> int:

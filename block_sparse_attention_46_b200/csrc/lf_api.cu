@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <string.h>
 
@@ -389,6 +391,51 @@ int noalloc_scratch(void** out) {
 
 // ===================================================================== C ABI
 extern "C" {
+
+int lf_cag_schedule(int32_t n_chunks, int32_t first, float mean_sparsity, float final_sparsity,
+                    const int32_t* n_hist, int32_t n_bpf, int32_t kf_max, float* keep,
+                    int32_t* k_f, int32_t* k_b) {
+  const bool budgets = n_hist != nullptr || k_f != nullptr || k_b != nullptr;
+  if (n_chunks < 1 || n_chunks > 4096 || first < 1 || first > n_chunks || keep == nullptr ||
+      n_bpf < 1 || kf_max < 1 || !(mean_sparsity >= 0.f && mean_sparsity < 1.f) ||
+      !(final_sparsity >= 0.f && final_sparsity < 1.f) ||
+      (budgets && (n_hist == nullptr || k_f == nullptr || k_b == nullptr)))
+    return LF_ERR_INVALID_ARG;
+  // mean over the sparse chunks of alpha_i = 1/sqrt(i), and alpha of the last chunk
+  double a_mean = 0.0;
+  for (int i = first; i <= n_chunks; ++i) a_mean += 1.0 / std::sqrt((double)i);
+  a_mean /= (double)(n_chunks - first + 1);
+  const double a_last = 1.0 / std::sqrt((double)n_chunks);
+  double beta = 0.0, s_base = final_sparsity;
+  if (first < n_chunks) {
+    // s_base - beta * a_mean = mean, s_base - beta * a_last = final
+    beta = ((double)final_sparsity - (double)mean_sparsity) / (a_mean - a_last);
+    s_base = (double)final_sparsity + beta * a_last;
+  } else if (std::fabs((double)mean_sparsity - (double)final_sparsity) > 1e-6) {
+    return LF_ERR_INVALID_ARG;
+  }
+  for (int i = 1; i <= n_chunks; ++i) {
+    double r = 1.0;
+    if (i >= first) r = std::min(1.0, std::max(0.0, 1.0 - (s_base - beta / std::sqrt((double)i))));
+    keep[i - 1] = (float)r;
+    if (!budgets) continue;
+    const int F = n_hist[i - 1];
+    if (F <= 0) {
+      k_f[i - 1] = k_b[i - 1] = 0;
+    } else if (i < first) {
+      k_f[i - 1] = F;
+      k_b[i - 1] = n_bpf;
+    } else {
+      const int kf = std::min(kf_max, F);
+      // halves round up; the 1e-9 keeps an exact half that arrives as x.4999999 from
+      // rounding in the keep ratio on the upper side
+      const int kb = (int)std::floor(r * F * n_bpf / kf + 0.5 + 1e-9);
+      k_f[i - 1] = kf;
+      k_b[i - 1] = std::min(n_bpf, std::max(1, kb));
+    }
+  }
+  return LF_OK;
+}
 
 int lf_abi_version(void) { return LF_ABI_VERSION; }
 

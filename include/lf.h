@@ -216,6 +216,23 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
  * 1e-4 for -125 <= x <= 8; x below -126 gives about 1.2e-38).  x, y: device fp32 [n]. */
 int lf_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 
+/* Chunk-aware growth of the sparsity [LF-gist 2.1, consistency-aware growth]: the sparsity
+ * of chunk i rises as the noise level alpha_i falls, s_i = s_base - alpha_i * beta, here
+ * with alpha_i = 1/sqrt(i).  Chunks first..n_chunks are sparse; beta and s_base are
+ * solved so that the mean of s_i over them is mean_sparsity and s_{n_chunks} is
+ * final_sparsity (first == n_chunks needs mean == final).  Host only, no device work.
+ * Outputs per chunk i = 1..n_chunks (HOST arrays of n_chunks entries):
+ *   keep[i-1] = 1 - s_i, clamped to [0, 1] (1 for chunks before `first`);
+ *   if n_hist, k_f and k_b are given, the top-k budget of a chunk with F = n_hist[i-1]
+ *   history frames of n_bpf blocks: (0, 0) when F = 0; (F, n_bpf) (dense) before
+ *   `first`; else k_f = min(kf_max, F), k_b = floor(keep * F * n_bpf / k_f + 1/2)
+ *   (halves round up) clamped to [1, n_bpf], so that k_f * k_b / (F * n_bpf) ~ keep.
+ * LF_ERR_INVALID_ARG for n_chunks outside [1, 4096], first outside [1, n_chunks],
+ * sparsities outside [0, 1), n_bpf or kf_max < 1, or missing outputs. */
+int lf_cag_schedule(int32_t n_chunks, int32_t first, float mean_sparsity, float final_sparsity,
+                    const int32_t* n_hist, int32_t n_bpf, int32_t kf_max, float* keep,
+                    int32_t* k_f, int32_t* k_b);
+
 /* Reads (synchronising the current device) and optionally clears the device status word
  * of the current device: LF_OK, LF_ERR_BAD_INDEX or LF_ERR_TIMEOUT.  Returns LF_ERR_CUDA
  * if the read itself fails. */
