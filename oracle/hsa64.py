@@ -173,6 +173,25 @@ def select_blocks(q_blk: np.ndarray, k_blk: np.ndarray, frame_idx: np.ndarray, k
 
 
 # --------------------------------------------------------------- (d) attention
+def select_blocks_1d(q_blk: np.ndarray, k_blk: np.ndarray, k: int):
+    """[LF-yly 四, the one-dimensional block-sparse ablation] No frame stage: each query
+    block keeps the k best-scoring history blocks over all frames (global id f * n_bpf + b,
+    equal scores to the lower id).  Returns block_idx [H, n_qb, min(k, F * n_bpf)] ascending
+    and the scores of every history block [H, n_qb, F * n_bpf]."""
+    H, nqb, _ = q_blk.shape
+    F, nbpf = k_blk.shape[1], k_blk.shape[2]
+    nb = F * nbpf
+    kk = min(k, nb)
+    idx = np.empty((H, nqb, kk), dtype=np.int64)
+    s = np.empty((H, nqb, nb))
+    for h in range(H):
+        for qb in range(nqb):
+            for f in range(F):
+                s[h, qb, f * nbpf:(f + 1) * nbpf] = block_scores_in_frame(q_blk[h, qb], k_blk[h, f])
+            idx[h, qb] = topk_lower_index(list(s[h, qb]), kk)
+    return idx, s
+
+
 def key_set(shape, qb_blocks: Sequence[int], cur_h: np.ndarray, cache_h: np.ndarray,
             hist_slots, sink_slots) -> np.ndarray:
     """Keys (or values) one query block attends to, in a fixed order: the whole current

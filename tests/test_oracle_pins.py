@@ -298,3 +298,37 @@ def test_executed_flops_counts_valid_pairs():
     r = O.forward_chunk(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
                         ci.hist_slots, ci.sink_slots)
     assert O.executed_flops(ci.shape, r["block_idx"]) == 4 * 16 * 2 * 100 * (100 + 50 + 150)
+
+
+# ------------------------------------------------------------------ 1-D ablation selection
+@pytest.mark.parametrize("seed", range(6))
+def test_select_blocks_1d_brute_force(seed):
+    """No frame stage: per query block the k-subset of ALL history blocks with the largest
+    score sum (scores recomputed here as plain dot products), ties to lower ids."""
+    g = np.random.default_rng(100 + seed)
+    H, nqb, F, nbpf, d = 2, 3, 3, 4, 8
+    q = g.standard_normal((H, nqb, d))
+    kb = g.standard_normal((H, F, nbpf, d))
+    if seed % 2:                       # exact ties: duplicated block keys across frames
+        kb[:, 2] = kb[:, 0]
+    k = int(g.integers(1, F * nbpf + 1))
+    idx, s = O.select_blocks_1d(q, kb, k)
+    assert idx.shape == (H, nqb, k)
+    for h in range(H):
+        for qq in range(nqb):
+            flat = [float(np.dot(q[h, qq], kb[h, f, b])) for f in range(F) for b in range(nbpf)]
+            assert np.allclose(s[h, qq], flat, rtol=0, atol=1e-12)
+            assert list(idx[h, qq]) == _brute_topk(flat, k)
+
+
+def test_select_blocks_1d_degenerate_and_two_stage():
+    g = np.random.default_rng(7)
+    q = g.standard_normal((1, 2, 4))
+    kb = g.standard_normal((1, 2, 3, 4))
+    idx, _ = O.select_blocks_1d(q, kb, 99)                 # k >= all blocks: every block
+    assert idx.tolist() == [[list(range(6)), list(range(6))]]
+    # with a single frame the frame stage is trivial: 1-D equals the two-stage selection
+    kb1 = kb[:, :1]
+    one_d, _ = O.select_blocks_1d(q, kb1, 2)
+    two, _ = O.select_blocks(q, kb1, np.zeros((1, 2, 1), dtype=np.int64), 2)
+    assert np.array_equal(one_d, two)
