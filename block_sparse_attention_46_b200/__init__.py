@@ -20,7 +20,7 @@ __all__ = [
     "lf_attn_workspace_size", "lf_forward_workspace_size", "lf_device_status",
     "lf_select_chunk", "lf_select_workspace_size", "lf_block_sparse_attn_noalloc",
     "lf_noalloc_scratch_bytes", "lf_pooled_cache_bytes", "lf_pool_frames",
-    "lf_select_chunk_cached", "lf_cag_schedule",
+    "lf_select_chunk_cached", "lf_cag_schedule", "lf_select_chunk_1d",
     "lf_status_string", "lf_abi_version", "derived", "LIB_PATH",
 ]
 
@@ -72,6 +72,7 @@ _SIGS = {
                                        ctypes.POINTER(ctypes.c_float), _I32P, _I32P]),
     "lf_pool_frames": (ctypes.c_int, [_SHP, _P, _I32P, ctypes.c_int32, _P, _P]),
     "lf_select_chunk_cached": (ctypes.c_int, [_SHP, _P, _P, _I32P, _P, _P, _SZ, _P]),
+    "lf_select_chunk_1d": (ctypes.c_int, [_SHP, _P, _P, _I32P, _P, _P, _SZ, _P]),
     "lf_block_sparse_attn_noalloc": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P,
                                                     _P, _P, _P]),
 }
@@ -183,6 +184,18 @@ def lf_select_chunk(shape, q, k_cache, hist_slots, block_idx, workspace=None, st
     _check(load().lf_select_chunk(ctypes.byref(sh), _ptr(q), _ptr(k_cache), hs, _ptr(block_idx),
                                   _ptr(workspace), workspace.numel(), _stream(stream)),
            "lf_select_chunk")
+
+
+def lf_select_chunk_1d(shape, q, k_cache, hist_slots, block_idx, workspace=None, stream=None):
+    """One-dimensional selection (no frame stage): the kf*kb best blocks over all frames."""
+    sh = make_shape(shape)
+    hs, _keep = _slots(hist_slots)
+    if workspace is None:
+        workspace = torch.empty(max(lf_select_workspace_size(shape), 256), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().lf_select_chunk_1d(ctypes.byref(sh), _ptr(q), _ptr(k_cache), hs,
+                                     _ptr(block_idx), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "lf_select_chunk_1d")
 
 
 def lf_pooled_cache_bytes(shape) -> int:

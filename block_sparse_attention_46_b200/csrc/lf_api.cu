@@ -601,6 +601,41 @@ int lf_select_chunk(const lf_shape* shape, const void* q, const void* k_cache,
   return run_select(D, q, k_cache, hist_slots, carve(D, workspace), block_idx, stream, &plans_ready);
 }
 
+int lf_select_chunk_1d(const lf_shape* shape, const void* q, const void* k_cache,
+                       const int32_t* hist_slots, int32_t* block_idx, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (D.F < 1) return LF_ERR_INVALID_ARG;
+  if (q == nullptr || k_cache == nullptr || block_idx == nullptr || !aligned(q, 16) ||
+      !aligned(k_cache, 16) || !aligned(block_idx, 4))
+    return LF_ERR_INVALID_ARG;
+  if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
+  const int nb = D.F * D.nbpf;
+  if (nb > lf::kFuseMaxBlocks) return LF_ERR_UNSUPPORTED;
+  const FwdWs need = carve(D, nullptr);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need.bytes)
+    return LF_ERR_WORKSPACE;
+  const FwdWs w = carve(D, workspace);
+  if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, nullptr, stream)) != LF_OK)
+    return rc;
+  lf::ScoreArgs sa{};
+  sa.q_blk = w.q_blk;
+  sa.k_blk = w.k_blk;
+  sa.k_pool = nullptr;
+  sa.scores = w.scores;
+  const dim3 sgrid(lf::cdiv(nb, lf::kScoreRows), D.H, lf::cdiv(D.nqb, lf::kScoreQb));
+  if (D.d == 128) lf::block_scores_kernel<128><<<sgrid, 256, 0, stream>>>(sa, D);
+  else lf::block_scores_kernel<64><<<sgrid, 256, 0, stream>>>(sa, D);
+  int n2 = 2;
+  while (n2 < nb) n2 <<= 1;
+  const size_t smem = (size_t)n2 * 3 * 4;
+  lf::select_topk_kernel<<<dim3(D.nqb, D.H), lf::kTopkThreads, smem, stream>>>(
+      w.scores, block_idx, D, n2);
+  return cuda_status(cudaGetLastError());
+}
+
 size_t lf_pooled_cache_bytes(const lf_shape* shape) {
   Dims D;
   if (make_dims(shape, &D) != LF_OK) return 0;

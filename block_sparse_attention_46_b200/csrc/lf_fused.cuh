@@ -182,4 +182,58 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
   }
 }
 
+// One-dimensional selection (no frame stage), the ablation the pages compare against
+// [LF-yly 四]: per (head, query block) the K = kf * kb best-scoring history blocks over all
+// frames, equal scores to the lower id, written in ascending id order.  One CTA per
+// (query block, head): a bitonic sort of the F * n_bpf scores (padded with -inf to n2, a
+// power of two) by (score descending, id ascending), then the first K ids are compacted
+// in id order by one warp.
+constexpr int kTopkThreads = 256;
+
+__global__ void __launch_bounds__(kTopkThreads)
+select_topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ block_idx,
+                   const Dims D, int n2) {
+  extern __shared__ float4 smt4[];
+  float* sv = reinterpret_cast<float*>(smt4);     // [n2] scores
+  int* si = reinterpret_cast<int*>(sv + n2);      // [n2] ids
+  int* mark = si + n2;                            // [n2] 1 = selected
+  const int qb = blockIdx.x, h = blockIdx.y;
+  const int nb = D.F * D.nbpf, K = D.nsel;
+  const float* src = scores + ((size_t)h * D.nqb + qb) * nb;
+  for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+    sv[i] = i < nb ? src[i] : -INFINITY;
+    si[i] = i;
+    mark[i] = 0;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < n2 / 2; t += blockDim.x) {
+        const int lo = 2 * t - (t & (stride - 1)), hi = lo + stride;
+        const float a = sv[lo], b = sv[hi];
+        const int ia = si[lo], ib = si[hi];
+        const bool a_first = a > b || (a == b && ia < ib);
+        if (a_first != ((lo & size) == 0)) {     // this bitonic run is built the other way
+          sv[lo] = b; sv[hi] = a;
+          si[lo] = ib; si[hi] = ia;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < K; i += blockDim.x) mark[si[i]] = 1;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int32_t* dst = block_idx + ((size_t)h * D.nqb + qb) * K;
+    int count = 0;
+    for (int base = 0; base < nb; base += 32) {
+      const bool sel = base + lane < nb && mark[base + lane];
+      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+      if (sel) dst[count + __popc(bal & ((1u << lane) - 1u))] = base + lane;
+      count += __popc(bal);
+    }
+  }
+}
+
 }  // namespace lf

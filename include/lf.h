@@ -9,7 +9,9 @@
  *             two-stage mask selection (frames, then blocks inside chosen frames),
  *             attention only on the chosen frame-block pairs.
  *   [LF-yly]  "南洋理工大学AI新突破 视频生成引擎模仿人脑高效学习" (m.youleyou.com),
- *             section 三 — the same three stages; frames retrieved by inner products.
+ *             section 三 — the same three stages; frames retrieved by inner products;
+ *             section 四 — the one-dimensional block-sparse attention it is compared with.
+ *   [LF-gist 2.1] the same explainer, section 2.1 — sparsity grown chunk by chunk.
  *   [SF]      Self Forcing article, rolling KV cache paragraph — cache of the last L
  *             frames, oldest evicted first.
  *   [RF]      "南洋理工大学突破：AI实现实时流式视频生成" (163.com, Rolling Forcing),
@@ -124,6 +126,18 @@ size_t lf_select_workspace_size(const lf_shape* shape);
 int lf_select_chunk(const lf_shape* shape, const void* q, const void* k_cache,
                     const int32_t* hist_slots, int32_t* block_idx, void* workspace,
                     size_t workspace_bytes, cudaStream_t stream);
+
+/* One-dimensional block selection, the ablation the pages compare the hierarchical
+ * selection with [LF-yly 四]: (a) pooling as in lf_select_chunk, then no frame stage:
+ * block_idx[h, qb] (device, [H, n_qb, kf*kb] with the effective kf = min(k_f, n_hist),
+ * kb = min(k_b, n_bpf)) receives the kf*kb history blocks with the largest scores
+ * q_blk . k_blk over ALL n_hist * n_bpf blocks, equal scores to the lower global id
+ * f*n_bpf + b, in ascending order -- the same layout lf_block_sparse_attn consumes.
+ * Same workspace as lf_select_chunk.  LF_ERR_UNSUPPORTED when n_hist * n_bpf > 2048.
+ * Requires n_hist >= 1. */
+int lf_select_chunk_1d(const lf_shape* shape, const void* q, const void* k_cache,
+                       const int32_t* hist_slots, int32_t* block_idx, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
 
 /* Pooled-key cache (incremental compression).  A frame's keys do not change once it is
  * in the KV cache [SF, rolling KV cache paragraph], so its block means [LF-gist 2.2,

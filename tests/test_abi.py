@@ -124,3 +124,15 @@ def test_pooled_cache_validation(lib):
     # the cache holds one fp32 row of d channels per (slot, head, block)
     s480 = W.p480_shape()
     assert lf.lf_pooled_cache_bytes(s480) == s480.n_slots * 12 * 25 * 128 * 4
+
+
+def test_select_1d_block_limit(lib):
+    # 40 history frames x 64 blocks = 2560 candidate blocks: beyond the 1-D selector
+    sh = lf.make_shape(_shape(H=1, T=4096, n_hist=40, n_slots=40))
+    hist, _k = _i32(list(range(40)))
+    assert lib.lf_select_chunk_1d(ctypes.byref(sh), FAKE, FAKE, hist, FAKE, FAKE, 1 << 40,
+                                  None) == 2
+    small = lf.make_shape(_shape())
+    h4, _k2 = _i32([0, 1, 2, 3])
+    assert lib.lf_select_chunk_1d(ctypes.byref(small), FAKE, FAKE, h4, FAKE, None, 0,
+                                  None) == 5
