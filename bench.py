@@ -128,6 +128,35 @@ def max_over_ranks(x: float, device) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(x: float, device) -> float:
+    """The sum of x over all ranks (work done by the whole job)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def head_shard(H: int, world: int, rank: int):
+    """Heads [h0, h1) of `rank` when H heads are split over `world` ranks: contiguous, the
+    first H % world ranks one head more.  Heads are independent at every stage, so a
+    sharded chunk needs no collective on the data path."""
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def shard_heads(ci, h0: int, h1: int):
+    """The chunk restricted to heads [h0, h1) (contiguous per-rank tensors)."""
+    from dataclasses import replace
+    part = lambda x: x[..., h0:h1, :].contiguous()
+    return replace(ci, shape=replace(ci.shape, H=h1 - h0), q=part(ci.q), k_cur=part(ci.k_cur),
+                   v_cur=part(ci.v_cur), k_cache=part(ci.k_cache), v_cache=part(ci.v_cache),
+                   planted=ci.planted[h0:h1])
+
+
 def weak_scaling_value(flops_per_rank: int, world: int, ms: float) -> float:
     """Whole-job TFLOP/s: every rank processed its own chunk in at most `ms`."""
     return world * flops_per_rank / (ms * 1e-3) / 1e12
@@ -268,7 +297,16 @@ def run_lf(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     lf.load()
-    ci, desc = make_workload(args.config, rank)
+    if args.shard == "heads":
+        # one chunk split by heads over the ranks (strong scaling): same seed everywhere
+        ci, desc = make_workload(args.config, 0)
+        h0, h1 = head_shard(ci.shape.H, world, rank)
+        if h1 <= h0:
+            raise SystemExit(f"--shard heads needs at most H={ci.shape.H} ranks")
+        ci = shard_heads(ci, h0, h1)
+        desc += f"; heads split over {world} ranks"
+    else:
+        ci, desc = make_workload(args.config, rank)
     sh = ci.shape
     nbpf, nqb, kf, kb = lf.derived(sh)
     t = {k: getattr(ci, k).to(dev) for k in ("q", "k_cur", "v_cur", "k_cache", "v_cache")}
@@ -354,7 +392,12 @@ def run_lf(args, rank, world, local_rank):
     step_ms = [a + b for a, b in zip(sel_ms, att_ms)]
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_step = total_ms / args.steps
-    value = weak_scaling_value(flops, world, ms_step)
+    if args.shard == "heads":
+        job_flops = sum_over_ranks(float(flops), dev)
+        value = job_flops / (ms_step * 1e-3) / 1e12
+    else:
+        job_flops = float(world * flops)
+        value = weak_scaling_value(flops, world, ms_step)
 
     # incremental compression: history block means kept per cache slot; per step the frames
     # that enter the cache (three slots re-pooled here, their keys unchanged, so the
@@ -401,6 +444,43 @@ def run_lf(args, rank, world, local_rank):
                "indices_equal_full_recompute": same,
                "api": "lf_pool_frames (the chunk's frames entering the cache) + "
                       "lf_select_chunk_cached, then lf_block_sparse_attn"}
+
+    # the one-dimensional ablation (no frame stage): its selection and the attention over
+    # the blocks it selects (the same number per query block, not clustered by frame)
+    abl = None
+    if sh.n_hist > 0 and sh.n_hist * -(-sh.T // sh.block) <= 2048:
+        bidx_1d = torch.empty_like(bidx)
+        out_1d = torch.empty_like(out)
+        ws_1d = torch.empty_like(ws)
+
+        def stages_1d():
+            lf.lf_select_chunk_1d(sh, t["q"], t["k_cache"], ci.hist_slots, bidx_1d, sws)
+            lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"],
+                                    t["v_cache"], ci.hist_slots, ci.sink_slots, bidx_1d,
+                                    out_1d, None, ws_1d)
+        for _ in range(3):
+            stages_1d()
+        torch.cuda.synchronize()
+        g_1d = torch.cuda.CUDAGraph()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g_1d, stream=cap):
+                stages_1d()
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+        ms_1d = []
+        for _ in range(max(3, min(args.steps, 200))):
+            flush_l2()
+            ev[0].record(stream)
+            g_1d.replay()
+            ev[1].record(stream)
+            ev[1].synchronize()
+            ms_1d.append(ev[0].elapsed_time(ev[1]))
+        f1d = executed_flops(sh, bidx_1d.cpu().numpy())
+        m1d = max_over_ranks(statistics.mean(ms_1d), dev)
+        abl = {"ms_per_step": m1d, "executed_gflop_per_chunk": f1d / 1e9,
+               "tflops": f1d / (m1d * 1e-3) / 1e12,
+               "api": "lf_select_chunk_1d + lf_block_sparse_attn"}
 
     # e2e through lf_forward_chunk with host buffers: every step copies its chunk's Q, K, V
     # from pinned host memory, runs the call, and copies the output back.  Two chunks are
@@ -463,7 +543,8 @@ def run_lf(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if args.shard == "heads" else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; per-frame key centroids, planted related frames)",
         "config": {"workload": desc,
                    "l2": "flushed before every timed step (256 MB written, then read back)",
@@ -480,12 +561,13 @@ def run_lf(args, rank, world, local_rank):
                                "unit": "GB/s", "frac": sel_gbs / pk["hbm_gbs"],
                                "kernels": "pool_blocks + block_scores + select_pick (lf_select_chunk)",
                                "peak_source": f"{src} hbm_gbs"},
-        "e2e": {"value": weak_scaling_value(flops, world, e2e_ms), "unit": "TFLOP/s",
+        "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "lf_forward_chunk per step, two chunks in flight (uploads, compute and "
                        "downloads on three streams)",
                 "output_equals_device_path": e2e_same},
         "incremental_compression": inc,
+        "ablation_1d": abl,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
@@ -507,6 +589,9 @@ def main():
     ap.add_argument("--impl", default="lf", choices=["lf", "reference"])
     ap.add_argument("--config", default="480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="chunks", choices=["chunks", "heads"],
+                    help="chunks: one chunk per rank (weak scaling); heads: one chunk split "
+                         "by heads over the ranks (strong scaling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

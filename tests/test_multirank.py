@@ -27,17 +27,20 @@ def _worker(rank, world, port, out):
         out[rank] = ms
         # every rank ran its own chunk: the whole-job value counts both
         out[2 + rank] = bench.weak_scaling_value(10 ** 12, world, ms)
+        # a head-sharded chunk: the job's work is the sum of the ranks' shares
+        out[4 + rank] = bench.sum_over_ranks([1.5e12, 2.5e12][rank], torch.device("cpu"))
     finally:
         dist.destroy_process_group()
 
 
 def test_two_gloo_ranks_take_max_and_count_all_work():
     world = 2
-    out = mp.get_context("spawn").Array("d", 4)
+    out = mp.get_context("spawn").Array("d", 6)
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world,
                        start_method="spawn", join=True)
     assert list(out[:2]) == [5.0, 5.0]
     assert out[2] == out[3] == pytest.approx(2 * 1e12 / 5e-3 / 1e12)
+    assert out[4] == out[5] == pytest.approx(4e12)
 
 
 def test_single_process_is_identity():
@@ -49,3 +52,22 @@ def test_tail_split_rule():
     import lf_workloads as W
     assert bench.tail_split(W.p480_shape())          # 456 tiles = 3 x 148 + 12
     assert not bench.tail_split(W.large_shape())     # 1560 tiles = 10 x 148 + 80
+
+
+@pytest.mark.parametrize("H,world", [(12, 1), (12, 2), (12, 5), (40, 8), (3, 3), (7, 4)])
+def test_head_shards_cover_every_head_once(H, world):
+    spans = [bench.head_shard(H, world, r) for r in range(world)]
+    assert spans[0][0] == 0 and spans[-1][1] == H
+    assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))          # contiguous
+    sizes = [h1 - h0 for h0, h1 in spans]
+    assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+
+
+def test_shard_heads_is_a_head_slice():
+    import lf_workloads as W
+    ci = W.tiny(0)
+    part = bench.shard_heads(ci, 1, 2)
+    assert part.shape.H == 1 and part.shape.T == ci.shape.T
+    assert torch.equal(part.q[:, 0], ci.q[:, 1])
+    assert torch.equal(part.k_cache[:, :, 0], ci.k_cache[:, :, 1])
+    assert part.q.is_contiguous() and part.hist_slots == ci.hist_slots
