@@ -248,7 +248,9 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   if (!plans_ready)
     lf::plan_kernel<<<dim3(lf::cdiv(lf::tile_count(D), lf::kPlanWarps), D.H), lf::kPlanWarps * 32, 0, st>>>(
         D.F > 0 ? block_idx : nullptr, w.plan, w.plan_cnt, D);
-  lf::schedule_kernel<<<1, 1024, 0, st>>>(w.plan_cnt, w.order, D);
+  const Split sp = make_split(D, n_sm);
+  lf::schedule_kernel<<<1, 1024, 0, st>>>(w.plan_cnt, w.order, D,
+                                          sp.n_tail > 0 ? sp.n_whole : lf::tile_count(D) * D.H);
   int rc = cuda_status(cudaGetLastError());
   if (rc != LF_OK) return rc;
 
@@ -270,7 +272,6 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   p.order = w.order;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  const Split sp = make_split(D, n_sm);
   p.tiles_per_head = lf::tile_count(D);
   p.n_whole = sp.n_whole;
   p.pieces = sp.pieces;

@@ -144,14 +144,19 @@ plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
 // ---------------------------------------------------------------------------------
 // Launch order of the tiles: longest first (list scheduling by decreasing cost, so the
 // last CTAs to start are the cheapest).  Cost = key tiles = dense tiles + sparse tiles;
-// a counting sort over the cost, stable in the tile index; one CTA of 1024 threads.
+// a counting sort over the cost; one CTA of 1024 threads.  Positions from split_pos on
+// are the tail tiles that run split into pieces: the tiles of the cost bucket that
+// straddles split_pos are placed in tile-index order, so the set of split tiles (and
+// with it the rounding of their outputs) is the same on every call; the order inside
+// any other bucket changes no result.
 // (Taking heads in groups of one wave, to keep the running CTAs' history blocks within
 // L2, measured no faster on the 480p chunk.)
 // ---------------------------------------------------------------------------------
 constexpr int kSchedBuckets = kMaxPlan + 1;
 
 __global__ void __launch_bounds__(1024)
-schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ order, const Dims D) {
+schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ order, const Dims D,
+                int split_pos) {
   __shared__ int hist[kSchedBuckets];
   __shared__ int start[kSchedBuckets];
   __shared__ int warp_tot[32];
@@ -197,23 +202,44 @@ schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ orde
       run += hist[k];
     }
   }
-  // stable placement: tiles with equal keys in tile-index order, so that the launch order
-  // (and with it which tiles form the split tail) is the same on every call
-  __shared__ int kbuf[1024];
+  // the bucket holding position split_pos (if the tail is split) goes in index order
+  __shared__ int kb_split, split_next, wpre[32];
+  if (threadIdx.x == 0) kb_split = -1;
+  __syncthreads();
+  for (int k = threadIdx.x; k < nb; k += blockDim.x)
+    if (start[k] <= split_pos && split_pos < start[k] + hist[k]) {
+      kb_split = k;
+      split_next = start[k];
+    }
+  __syncthreads();
   for (int base = 0; base < ntot; base += blockDim.x) {
     const int i = base + threadIdx.x;
     const int k = i < ntot ? key(i) : -1;
-    kbuf[threadIdx.x] = k;
+    const bool ordered = i < ntot && k == kb_split;
+    const uint32_t bal = __ballot_sync(0xffffffffu, ordered);
+    if (lane == 0) wpre[w] = __popc(bal);
     __syncthreads();
-    if (i < ntot) {
-      int rank = 0;
-      for (int j = 0; j < (int)threadIdx.x; ++j) rank += kbuf[j] == k;
-      order[start[k] + rank] = i;
+    if (w == 0) {                                  // exclusive prefix over the warps
+      const int x = lane < (int)(blockDim.x >> 5) ? wpre[lane] : 0;
+      int inc = x;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += y;
+      }
+      wpre[lane] = inc - x;
+      if (lane == 31) warp_tot[0] = inc;           // ordered tiles in this chunk
     }
     __syncthreads();
-    if (i < ntot) atomicAdd(&start[k], 1);
+    if (ordered)
+      order[split_next + wpre[w] + __popc(bal & ((1u << lane) - 1u))] = i;
+    else if (i < ntot)
+      order[atomicAdd(&start[k], 1)] = i;
+    __syncthreads();
+    if (threadIdx.x == 0) split_next += warp_tot[0];
     __syncthreads();
   }
+}
+
 }
 
 // ---------------------------------------------------------------------------------
