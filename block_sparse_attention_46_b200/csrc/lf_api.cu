@@ -185,7 +185,7 @@ Split make_split(const Dims& D, int n_sm) {
 #endif
   if (R == 0 || 2 * R > n_sm) return sp;
   int p = n_sm / R;
-  p = p < 16 ? p : 16;
+  p = p < lf::kMaxPieces ? p : lf::kMaxPieces;
   const int n_dense = lf::cdiv(D.ncur, 128);      // every tile has at least this many
   p = p < n_dense ? p : n_dense;
   if (p < 2) return sp;

@@ -240,8 +240,6 @@ schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ orde
   }
 }
 
-}
-
 // ---------------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------------
@@ -773,6 +771,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
 // m = max_k m_k, l = sum_k 2^(m_k - m) l_k, O = sum_k 2^(m_k - m) O_k / l.
 // CTA = (tail tile, group of kMergeRows rows); one thread per (row, 4 channels).
 constexpr int kMergeRows = 8;
+constexpr int kMaxPieces = 16;     // key ranges a tail tile is split into, at most
 
 __global__ void __launch_bounds__(256)
 merge_kernel(const AttnParams P, const Dims D, int HD) {
@@ -789,19 +788,33 @@ merge_kernel(const AttnParams P, const Dims D, int HD) {
     else { qb = qbA; i = r; }
     if (qb < 0 || i >= block_len(D, qb % D.nbpf)) continue;
     const int tok = (qb / D.nbpf) * D.T + (qb % D.nbpf) * D.B + i;
+    // every piece's state loaded at once (the loads are independent), then combined in
+    // piece order
+    float mk[kMaxPieces], lk[kMaxPieces];
+    float4 xk[kMaxPieces];
+#pragma unroll
+    for (int k = 0; k < kMaxPieces; ++k) {
+      mk[k] = -INFINITY;
+      lk[k] = 0.f;
+      xk[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k < P.pieces) {
+        const size_t unit = (size_t)tail * P.pieces + k;
+        mk[k] = P.part_ml[(unit * 2) * 128 + r];
+        lk[k] = P.part_ml[(unit * 2 + 1) * 128 + r];
+        xk[k] = reinterpret_cast<const float4*>(P.part_o + (unit * 128 + r) * HD)[c4];
+      }
+    }
     float m = -INFINITY;
-    for (int k = 0; k < P.pieces; ++k)
-      m = fmaxf(m, P.part_ml[((size_t)(tail * P.pieces + k) * 2) * 128 + r]);
+#pragma unroll
+    for (int k = 0; k < kMaxPieces; ++k) m = fmaxf(m, mk[k]);
     float l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < P.pieces; ++k) {
-      const int unit = tail * P.pieces + k;
-      const float mk = P.part_ml[((size_t)unit * 2) * 128 + r];
-      if (mk == -INFINITY) continue;
-      const float w = exp2f(mk - m);
-      l += w * P.part_ml[((size_t)unit * 2 + 1) * 128 + r];
-      const float4 x = reinterpret_cast<const float4*>(P.part_o + ((size_t)unit * 128 + r) * HD)[c4];
-      o.x += w * x.x; o.y += w * x.y; o.z += w * x.z; o.w += w * x.w;
+#pragma unroll
+    for (int k = 0; k < kMaxPieces; ++k) {
+      if (mk[k] == -INFINITY) continue;          // a piece with no valid key (or past P.pieces)
+      const float w = exp2f(mk[k] - m);
+      l += w * lk[k];
+      o.x += w * xk[k].x; o.y += w * xk[k].y; o.z += w * xk[k].z; o.w += w * xk[k].w;
     }
     const float inv = 1.0f / l;
     __nv_bfloat162 a = __floats2bfloat162_rn(o.x * inv, o.y * inv);
