@@ -20,5 +20,7 @@ def gpu_lib():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import block_sparse_attention_46_b200 as lf
+    from block_sparse_attention_46_b200 import build
+    build.build()      # rebuilds if a source is newer than liblf.so; raises if nvcc fails
     lf.load()          # raises if liblf.so is absent or does not load
     return lf
