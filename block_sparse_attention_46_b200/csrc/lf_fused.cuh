@@ -13,7 +13,7 @@
 namespace lf {
 
 #ifndef LF_FUSE_QB
-#define LF_FUSE_QB 8
+#define LF_FUSE_QB 2
 #endif
 #ifndef LF_SCORE_QB
 #define LF_SCORE_QB 16
@@ -131,9 +131,10 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
   __syncthreads();
 
   const float invT = 1.0f / (float)D.T;
-  for (int g = warp; g < kFuseQb; g += blockDim.x / 32) {
-    const int qb = qb0 + g;
-    if (qb >= D.nqb) continue;
+  const int nwarps = blockDim.x / 32;
+  // frame scores (by linearity from the block scores) and frame top-k: a warp per query block
+  for (int g = warp; g < kFuseQb; g += nwarps) {
+    if (qb0 + g >= D.nqb) continue;
     const float* s = sc + (size_t)g * NB;
     float fs[kMaxPerLane];
 #pragma unroll
@@ -149,23 +150,29 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
     }
     const uint32_t taken = warp_topk(fs, D.F, D.kf);
     warp_write_ascending(taken, D.F, sf + g * D.kf, 0);
-    __syncwarp();
-    for (int j = 0; j < D.kf; ++j) {
-      const int f = sf[g * D.kf + j];
-      float bs[kMaxPerLane];
-#pragma unroll
-      for (int u = 0; u < kMaxPerLane; ++u) {
-        const int b = lane + 32 * u;
-        bs[u] = b < D.nbpf ? s[f * D.nbpf + b] : -INFINITY;
-      }
-      const uint32_t tb = warp_topk(bs, D.nbpf, D.kb);
-      warp_write_ascending(tb, D.nbpf, sl + g * D.nsel + j * D.kb, f * D.nbpf);
-    }
-    __syncwarp();
-    int32_t* dst = block_idx + ((size_t)h * D.nqb + qb) * D.nsel;
-    for (int i = lane; i < D.nsel; i += 32) dst[i] = sl[g * D.nsel + i];
   }
   __syncthreads();
+  // block top-k inside each chosen frame: a warp per (query block, chosen frame)
+  for (int task = warp; task < kFuseQb * D.kf; task += nwarps) {
+    const int g = task / D.kf, j = task % D.kf;
+    if (qb0 + g >= D.nqb) continue;
+    const float* s = sc + (size_t)g * NB;
+    const int f = sf[g * D.kf + j];
+    float bs[kMaxPerLane];
+#pragma unroll
+    for (int u = 0; u < kMaxPerLane; ++u) {
+      const int b = lane + 32 * u;
+      bs[u] = b < D.nbpf ? s[f * D.nbpf + b] : -INFINITY;
+    }
+    const uint32_t tb = warp_topk(bs, D.nbpf, D.kb);
+    warp_write_ascending(tb, D.nbpf, sl + g * D.nsel + j * D.kb, f * D.nbpf);
+  }
+  __syncthreads();
+  // the lists (chosen frames ascending, blocks ascending inside each): all threads
+  for (int i = threadIdx.x; i < kFuseQb * D.nsel; i += blockDim.x) {
+    const int g = i / D.nsel, qb = qb0 + g;
+    if (qb < D.nqb) block_idx[((size_t)h * D.nqb + qb) * D.nsel + i % D.nsel] = sl[i];
+  }
 
   // key plans of the group's tiles (one warp per tile)
   const int ntiles = tile_count(D);
