@@ -1,11 +1,17 @@
-"""Chunk-aware sparsity growth (lf_cag_schedule, host only) against its closed form and
-against the growth-sweep workload's keep ratios and top-k budgets."""
+"""Chunk-aware sparsity growth (lf_cag_schedule, host only) against its closed form, the
+float64 oracle, the stored growth schedule under tests/golden, and the growth-sweep
+workload's keep ratios and top-k budgets."""
+import json
 import math
+import os
 
 import pytest
 
 import block_sparse_attention_46_b200 as lf
 import lf_workloads as W
+from oracle import cag64 as C
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "cag_growth_480p.json")
 
 
 @pytest.fixture(scope="module")
@@ -13,6 +19,34 @@ def lib():
     from block_sparse_attention_46_b200 import build
     build.build()
     return lf.load()
+
+
+def test_growth_golden(lib):
+    """The stored 7-chunk schedule (80% mean over chunks 2-7, 90% at chunk 7)."""
+    g = json.load(open(GOLDEN))
+    a = g["args"]
+    keep, kf, kb = lf.lf_cag_schedule(a["n_chunks"], a["first"], a["mean_sparsity"],
+                                      a["final_sparsity"], a["n_hist"], n_bpf=a["n_bpf"],
+                                      kf_max=a["kf_max"])
+    assert keep == pytest.approx(g["keep"], abs=1e-6)        # float32 outputs
+    assert [list(p) for p in zip(kf, kb)] == g["budgets"]
+    # the workload's 4-decimal keep ratios and its budgets are the stored ones
+    assert W.GROWTH_KEEP == [round(v, 4) for v in g["keep"]]
+    assert [list(p) for p in W.GROWTH_TOPK] == g["budgets"]
+
+
+@pytest.mark.parametrize("n,first,mean,final,n_bpf,kf_max",
+                         [(7, 2, 0.8, 0.9, 25, 6), (20, 2, 0.8, 0.95, 25, 6),
+                          (12, 3, 0.6, 0.85, 13, 4), (5, 1, 0.3, 0.2, 7, 3),
+                          (9, 4, 0.9, 0.97, 100, 8)])
+def test_matches_oracle(lib, n, first, mean, final, n_bpf, kf_max):
+    n_hist = [min(3 * i, 21) for i in range(n)]
+    keep, kf, kb = lf.lf_cag_schedule(n, first, mean, final, n_hist, n_bpf=n_bpf,
+                                      kf_max=kf_max)
+    keep_o, budgets_o = C.cag_schedule(n, first, mean, final, n_hist, n_bpf=n_bpf,
+                                       kf_max=kf_max)
+    assert keep == pytest.approx(keep_o, abs=1e-6)
+    assert list(zip(kf, kb)) == budgets_o
 
 
 def test_growth_sweep_schedule(lib):

@@ -14,7 +14,10 @@ the method reduces to, and invariants the method's description implies:
   torch's scaled_dot_product_attention in float64; zero queries give the uniform
   average of the key set's values and lse = log(|key set|); probabilities are
   non-negative and sum to one; unselected keys can be permuted or replaced freely;
-* fixed complexity: the number of selected blocks does not depend on the history length.
+* fixed complexity: the number of selected blocks does not depend on the history length;
+* chunk-aware growth: the two conditions that fix (s_base, beta) hold, a two-chunk case
+  solved by hand, constant sparsity when the mean and the final level agree, growth with
+  the chunk index, and budgets against an exhaustive search over (k_f, k_b) pairs.
 """
 import itertools
 import math
@@ -24,6 +27,7 @@ import pytest
 import torch
 
 import lf_workloads as W
+from oracle import cag64 as C
 from oracle import hsa64 as O
 
 
@@ -332,3 +336,56 @@ def test_select_blocks_1d_degenerate_and_two_stage():
     one_d, _ = O.select_blocks_1d(q, kb1, 2)
     two, _ = O.select_blocks(q, kb1, np.zeros((1, 2, 1), dtype=np.int64), 2)
     assert np.array_equal(one_d, two)
+
+
+# ------------------------------------------------------------------ chunk-aware growth
+@pytest.mark.parametrize("n,first,mean,final", [(7, 2, 0.8, 0.9), (20, 2, 0.8, 0.95),
+                                                (5, 3, 0.5, 0.6), (4, 1, 0.3, 0.2)])
+def test_cag_conditions_hold(n, first, mean, final):
+    """The solved schedule meets both conditions and has the form base - beta/sqrt(i)."""
+    s, s_base, beta = C.cag_sparsity(n, first, mean, final)
+    sparse = s[first - 1:]
+    assert sum(sparse) / len(sparse) == pytest.approx(mean, abs=1e-12)
+    assert s[-1] == pytest.approx(final, abs=1e-12)
+    assert all(v == 0.0 for v in s[:first - 1])
+    for i in range(first, n + 1):
+        assert s[i - 1] == pytest.approx(s_base - beta / math.sqrt(i), abs=1e-12)
+    # later chunks are sparser exactly when the last chunk is above the mean
+    steps = [b - a for a, b in zip(sparse, sparse[1:])]
+    assert all((d > 0) == (final > mean) for d in steps)
+
+
+def test_cag_two_chunks_by_hand():
+    """n = 2, first = 1: (s_1 + s_2)/2 = m and s_2 = f give s_1 = 2m - f, and
+    beta = (s_2 - s_1) / (1 - 1/sqrt(2))."""
+    m, f = 0.5, 0.7
+    s, s_base, beta = C.cag_sparsity(2, 1, m, f)
+    assert s == pytest.approx([2 * m - f, f], abs=1e-12)
+    assert beta == pytest.approx((f - (2 * m - f)) / (1 - 1 / math.sqrt(2)), abs=1e-12)
+    assert s_base == pytest.approx(s[0] + beta, abs=1e-12)
+
+
+def test_cag_constant_and_single_sparse_chunk():
+    s, _, beta = C.cag_sparsity(6, 2, 0.75, 0.75)
+    assert beta == pytest.approx(0.0, abs=1e-12)
+    assert s[1:] == pytest.approx([0.75] * 5, abs=1e-12)
+    s, _, beta = C.cag_sparsity(3, 3, 0.4, 0.4)
+    assert s == [0.0, 0.0, 0.4] and beta == 0.0
+    with pytest.raises(ValueError):
+        C.cag_sparsity(3, 3, 0.4, 0.5)
+    keep, budgets = C.cag_schedule(3, 2, 0.5, 0.5, [0, 4, 4], n_bpf=10, kf_max=2)
+    assert keep == [1.0, 0.5, 0.5] and budgets[0] == (0, 0)
+
+
+@pytest.mark.parametrize("F,n_bpf,kf_max", [(3, 25, 6), (18, 25, 6), (5, 13, 2), (1, 4, 8)])
+def test_cag_budget_exhaustive(F, n_bpf, kf_max):
+    """Over every pair k_f in [1, kf_max], k_b in [1, n_bpf], the budget keeps
+    k_f = min(kf_max, F) frames and its k_b brings the kept fraction nearest to the keep
+    ratio among all k_b for that k_f; it never exceeds the frame's blocks."""
+    for keep in np.linspace(0.0, 1.0, 41):
+        kf, kb = C.cag_budget(float(keep), F, n_bpf, kf_max, dense=False)
+        assert kf == min(kf_max, F) and 1 <= kb <= n_bpf
+        errs = {b: abs(kf * b / (F * n_bpf) - keep) for b in range(1, n_bpf + 1)}
+        assert errs[kb] <= min(errs.values()) + 1e-12
+        assert C.cag_budget(float(keep), F, n_bpf, kf_max, dense=True) == (F, n_bpf)
+    assert C.cag_budget(0.5, 0, n_bpf, kf_max, dense=False) == (0, 0)
