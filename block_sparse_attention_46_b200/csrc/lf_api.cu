@@ -315,6 +315,18 @@ FwdWs carve(const Dims& D, void* base) {
 
 // Block scores (from the per-call pooled keys w.k_blk, or from the pooled-key cache k_pool
 // through hist_slots) and the pick kernel (frame and block top-k, key plans).
+// Scores of every history block against every pooled query block into sa.scores.
+int launch_block_scores(const Dims& D, const lf::ScoreArgs& sa, cudaStream_t stream) {
+  const dim3 grid(lf::cdiv(D.F * D.nbpf, lf::kScoreRows), D.H, lf::cdiv(D.nqb, lf::kScoreQb));
+  auto kern = D.d == 128 ? lf::block_scores_kernel<128> : lf::block_scores_kernel<64>;
+  const size_t smem = D.d == 128 ? lf::score_smem<128>() : lf::score_smem<64>();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LF_ERR_CUDA;
+  kern<<<grid, lf::kScoreThreads, smem, stream>>>(sa, D);
+  return cuda_status(cudaGetLastError());
+}
+
 int launch_scores_pick(const Dims& D, const FwdWs& w, const float* k_pool,
                        const int32_t* hist_slots, const AttnWs& aw, int32_t* bidx,
                        cudaStream_t stream) {
@@ -325,15 +337,14 @@ int launch_scores_pick(const Dims& D, const FwdWs& w, const float* k_pool,
   sa.scores = w.scores;
   if (k_pool != nullptr)
     for (int f = 0; f < D.F; ++f) sa.slots[f] = hist_slots[f];
-  const dim3 sgrid(lf::cdiv(D.F * D.nbpf, lf::kScoreRows), D.H, lf::cdiv(D.nqb, lf::kScoreQb));
-  if (D.d == 128) lf::block_scores_kernel<128><<<sgrid, 256, 0, stream>>>(sa, D);
-  else lf::block_scores_kernel<64><<<sgrid, 256, 0, stream>>>(sa, D);
+  int rc = launch_block_scores(D, sa, stream);
+  if (rc != LF_OK) return rc;
   const size_t smem = lf::fused_select_smem(D);
   if (cudaFuncSetAttribute(lf::select_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return LF_ERR_CUDA;
-  lf::select_pick_kernel<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), 256, smem, stream>>>(
-      w.scores, bidx, aw.plan, aw.plan_cnt, D);
+  lf::select_pick_kernel<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), lf::kPickThreads, smem,
+                           stream>>>(w.scores, bidx, aw.plan, aw.plan_cnt, D);
   return cuda_status(cudaGetLastError());
 }
 
@@ -626,9 +637,7 @@ int lf_select_chunk_1d(const lf_shape* shape, const void* q, const void* k_cache
   sa.k_blk = w.k_blk;
   sa.k_pool = nullptr;
   sa.scores = w.scores;
-  const dim3 sgrid(lf::cdiv(nb, lf::kScoreRows), D.H, lf::cdiv(D.nqb, lf::kScoreQb));
-  if (D.d == 128) lf::block_scores_kernel<128><<<sgrid, 256, 0, stream>>>(sa, D);
-  else lf::block_scores_kernel<64><<<sgrid, 256, 0, stream>>>(sa, D);
+  if ((rc = launch_block_scores(D, sa, stream)) != LF_OK) return rc;
   int n2 = 2;
   while (n2 < nb) n2 <<= 1;
   const size_t smem = (size_t)n2 * 3 * 4;

@@ -15,9 +15,6 @@ namespace lf {
 #ifndef LF_FUSE_QB
 #define LF_FUSE_QB 2
 #endif
-#ifndef LF_SCORE_QB
-#define LF_SCORE_QB 16
-#endif
 constexpr int kFuseQb = LF_FUSE_QB;        // query blocks per CTA (even: whole tile pairs)
 constexpr int kFuseMaxBlocks = 2048;       // F * n_bpf handled by the fused path
 constexpr int kFuseMaxSel = 256;           // k_f * k_b handled by the fused path
@@ -33,13 +30,18 @@ __host__ __device__ inline size_t fused_select_smem(const Dims& D) {
 }
 
 // Scores of every history block against every pooled query block of head h:
-// s[h, qb, r] = q_blk[h, qb] . k_blk[h, r], r = f * n_bpf + b.  CTA = (64 rows, head,
-// kScoreQb query blocks); rows and queries are staged in shared memory with coalesced
-// loads; thread (row, quarter) computes kScoreQb / 4 query blocks against one row, each
-// score one fixed-order sum over the channels.
-constexpr int kScoreRows = 64, kScoreQb = LF_SCORE_QB;
-constexpr int kScoreQpt = kScoreQb * kScoreRows / 256;    // query blocks per thread
-static_assert(kScoreQpt >= 1 && kScoreQpt * 256 == kScoreQb * kScoreRows, "score tiling");
+// s[h, qb, r] = q_blk[h, qb] . k_blk[h, r], r = f * n_bpf + b.  CTA = (128 rows, head,
+// 16 query blocks), four warps; rows and queries are staged in shared memory with
+// coalesced loads and a row pitch of d + 4 floats.  Each thread computes a 4 x 4 tile,
+// rows rg + 8i and query blocks qg + 4u (rg = lane % 8, qg = lane / 8): at every step the
+// warp reads 8 distinct rows and 4 distinct queries, one 128-byte wavefront each, so the
+// loop runs at the FMA rate.  Each score is one fixed-order sum over the channels.
+constexpr int kScoreRows = 128, kScoreQb = 16, kScoreThreads = 128;
+
+template <int HD>
+__host__ __device__ constexpr size_t score_smem() {
+  return (size_t)(kScoreRows + kScoreQb) * (HD / 4 + 1) * sizeof(float4);
+}
 
 struct ScoreArgs {
   const float* q_blk;   // [H, nqb, d]
@@ -50,70 +52,93 @@ struct ScoreArgs {
 };
 
 template <int HD>
-__global__ void __launch_bounds__(256)   // staging assumes exactly 256 threads
+__global__ void __launch_bounds__(kScoreThreads)   // staging assumes exactly 128 threads
 block_scores_kernel(const __grid_constant__ ScoreArgs a, const Dims D) {
-  const float* __restrict__ q_blk = a.q_blk;
-  float* __restrict__ scores = a.scores;
-  __shared__ float4 sk4[kScoreRows * (HD / 4 + 1)];
-  __shared__ float4 sq4[kScoreQb * (HD / 4)];
+  constexpr int P = HD / 4 + 1;                        // float4 pitch, padded
+  extern __shared__ float4 smq4[];
+  float4* sk4 = smq4;                                  // [kScoreRows][P]
+  float4* sq4 = smq4 + kScoreRows * P;                 // [kScoreQb][P]
   const int NB = D.F * D.nbpf;
   const int r0 = blockIdx.x * kScoreRows, h = blockIdx.y, q0 = blockIdx.z * kScoreQb;
-  const int pitch = HD / 4 + 1;                       // float4 pitch, padded
   {
-    // kScoreRows * HD / 4 float4 = 2048 (d = 128): eight loads in flight per thread
-    constexpr int n4 = kScoreRows * (HD / 4);
-    float4 v[n4 / 256];
+    // kScoreRows * HD / 4 float4 (4096 at d = 128), eight loads in flight per thread
+    constexpr int n4 = kScoreRows * (HD / 4), batch = 8;
+    static_assert(n4 % (batch * kScoreThreads) == 0, "score staging");
+#pragma unroll 1
+    for (int i0 = 0; i0 < n4; i0 += batch * kScoreThreads) {
+      float4 v[batch];
 #pragma unroll
-    for (int u = 0; u < n4 / 256; ++u) {
-      const int i = threadIdx.x + u * 256, r = i / (HD / 4), c4 = i % (HD / 4);
-      const int rr = r0 + r;
-      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (rr < NB) {
-        const float* row = a.k_pool != nullptr
-            ? a.k_pool + (((size_t)a.slots[rr / D.nbpf] * D.H + h) * D.nbpf + rr % D.nbpf) * HD
-            : a.k_blk + ((size_t)h * NB + rr) * HD;
-        v[u] = __ldg(reinterpret_cast<const float4*>(row) + c4);
+      for (int u = 0; u < batch; ++u) {
+        const int i = i0 + threadIdx.x + u * kScoreThreads, r = i / (HD / 4), c4 = i % (HD / 4);
+        const int rr = r0 + r;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (rr < NB) {
+          const float* row = a.k_pool != nullptr
+              ? a.k_pool + (((size_t)a.slots[rr / D.nbpf] * D.H + h) * D.nbpf + rr % D.nbpf) * HD
+              : a.k_blk + ((size_t)h * NB + rr) * HD;
+          v[u] = __ldg(reinterpret_cast<const float4*>(row) + c4);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < batch; ++u) {
+        const int i = i0 + threadIdx.x + u * kScoreThreads, r = i / (HD / 4), c4 = i % (HD / 4);
+        sk4[r * P + c4] = v[u];
       }
     }
-#pragma unroll
-    for (int u = 0; u < n4 / 256; ++u) {
-      const int i = threadIdx.x + u * 256, r = i / (HD / 4), c4 = i % (HD / 4);
-      sk4[r * pitch + c4] = v[u];
-    }
   }
-  for (int i = threadIdx.x; i < kScoreQb * (HD / 4); i += 256) {
+  for (int i = threadIdx.x; i < kScoreQb * (HD / 4); i += kScoreThreads) {
     const int g = i / (HD / 4), c4 = i % (HD / 4);
-    sq4[i] = q0 + g < D.nqb
-        ? __ldg(reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + q0 + g) * HD) + c4)
+    sq4[g * P + c4] = q0 + g < D.nqb
+        ? __ldg(reinterpret_cast<const float4*>(a.q_blk + ((size_t)h * D.nqb + q0 + g) * HD) + c4)
         : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
-  const int r = threadIdx.x % kScoreRows, gq = threadIdx.x / kScoreRows;   // 4 quarters
-  float acc[kScoreQpt];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rg = lane & 7, qg = lane >> 3;
+  const int rb = warp * 32 + rg;                       // rows rb + 8i, i < 4
+  float acc[4][4];
 #pragma unroll
-  for (int u = 0; u < kScoreQpt; ++u) acc[u] = 0.f;
-#pragma unroll 8
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[u][i] = 0.f;
+#pragma unroll 4
   for (int c4 = 0; c4 < HD / 4; ++c4) {
-    const float4 k = sk4[r * pitch + c4];
+    float4 k[4], q[4];
 #pragma unroll
-    for (int u = 0; u < kScoreQpt; ++u) {
-      const float4 q = sq4[(gq * kScoreQpt + u) * (HD / 4) + c4];
-      acc[u] = fmaf(q.x, k.x, acc[u]); acc[u] = fmaf(q.y, k.y, acc[u]);
-      acc[u] = fmaf(q.z, k.z, acc[u]); acc[u] = fmaf(q.w, k.w, acc[u]);
+    for (int i = 0; i < 4; ++i) k[i] = sk4[(rb + 8 * i) * P + c4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) q[u] = sq4[(qg + 4 * u) * P + c4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float t = acc[u][i];
+        t = fmaf(q[u].x, k[i].x, t); t = fmaf(q[u].y, k[i].y, t);
+        t = fmaf(q[u].z, k[i].z, t); t = fmaf(q[u].w, k[i].w, t);
+        acc[u][i] = t;
+      }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int qb = q0 + qg + 4 * u;
+    if (qb >= D.nqb) continue;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = r0 + rb + 8 * i;
+      if (r < NB) a.scores[((size_t)h * D.nqb + qb) * NB + r] = acc[u][i];
     }
   }
-  if (r0 + r < NB)
-#pragma unroll
-    for (int u = 0; u < kScoreQpt; ++u) {
-      const int qb = q0 + gq * kScoreQpt + u;
-      if (qb < D.nqb) scores[((size_t)h * D.nqb + qb) * NB + r0 + r] = acc[u];
-    }
 }
 
 // Per (head, group of kFuseQb query blocks): frame scores by linearity from the block
 // scores, frame top-k, block top-k in each chosen frame, block_idx, and the key plans of
-// the group's query tiles.
-__global__ void __launch_bounds__(256)
+// the group's query tiles.  A tile's plan is written by the whole CTA from two bitmaps
+// over the F * n_bpf history blocks (one per query block of the tile): the union's bits
+// in id order give the entries, a prefix count of the union's words their positions.
+constexpr int kPickThreads = 256;
+constexpr int kFuseWords = kFuseMaxBlocks / 32;
+
+__global__ void __launch_bounds__(kPickThreads)
 select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block_idx,
                    uint32_t* __restrict__ plan, int32_t* __restrict__ plan_cnt, const Dims D) {
   extern __shared__ float4 sm4[];
@@ -174,18 +199,54 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
     if (qb < D.nqb) block_idx[((size_t)h * D.nqb + qb) * D.nsel + i % D.nsel] = sl[i];
   }
 
-  // key plans of the group's tiles (one warp per tile)
+  // key plans of the group's tiles
+  __shared__ uint32_t s_bits[2][kFuseWords];   // blocks chosen by the tile's query blocks
+  __shared__ int s_pre[kFuseWords];            // union entries in the words below
   const int ntiles = tile_count(D);
   const int per = D.B == 64 ? 2 : 1;                       // query blocks per tile
-  for (int p = warp; p < kFuseQb / per; p += blockDim.x / 32) {
+  const int nw = cdiv(NB, 32), nsink = D.S * D.nbpf;
+  for (int p = 0; p < kFuseQb / per; ++p) {
     const int qa = qb0 + p * per;
-    if (qa >= D.nqb) continue;
+    if (qa >= D.nqb) break;                                // the same for the whole CTA
     const int t = qa / per;
-    const bool two = per == 2 && qa + 1 < D.nqb;
-    const int cnt = warp_write_plan(sl + (qa - qb0) * D.nsel, D.nsel,
-                                    two ? sl + (qa + 1 - qb0) * D.nsel : sl, two ? D.nsel : 0,
-                                    plan + ((size_t)h * ntiles + t) * plan_stride(D), D);
-    if (lane == 0) plan_cnt[(size_t)h * ntiles + t] = cnt;
+    const int nq = (per == 2 && qa + 1 < D.nqb) ? 2 : 1;
+    for (int i = threadIdx.x; i < 2 * kFuseWords; i += blockDim.x) s_bits[i / kFuseWords][i % kFuseWords] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nq * D.nsel; i += blockDim.x) {
+      const int which = i / D.nsel;
+      const int id = sl[(qa - qb0 + which) * D.nsel + i % D.nsel];   // < NB by construction
+      atomicOr(&s_bits[which][id >> 5], 1u << (id & 31));
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+      for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        const int own = w < nw ? __popc(s_bits[0][w] | s_bits[1][w]) : 0;
+        int inc = own;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += v;
+        }
+        if (w < nw) s_pre[w] = carry + inc - own;
+        carry += __shfl_sync(0xffffffffu, inc, 31);
+      }
+      if (lane == 0) plan_cnt[(size_t)h * ntiles + t] = nsink + carry;
+    }
+    __syncthreads();
+    uint32_t* out = plan + ((size_t)h * ntiles + t) * plan_stride(D);
+    for (int e = threadIdx.x; e < nsink; e += blockDim.x) out[e] = plan_pack(e / D.nbpf, e % D.nbpf, 3u);
+    for (int x = threadIdx.x; x < NB; x += blockDim.x) {
+      const int w = x >> 5;
+      const uint32_t bit = 1u << (x & 31), ba = s_bits[0][w], bb = s_bits[1][w];
+      if ((ba | bb) & bit) {
+        const int pos = s_pre[w] + __popc((ba | bb) & (bit - 1u));
+        out[nsink + pos] = plan_pack(D.S + x / D.nbpf, x % D.nbpf,
+                                     ((ba & bit) ? 1u : 0u) | ((bb & bit) ? 2u : 0u));
+      }
+    }
+    __syncthreads();                                       // the bitmaps are reused
   }
 }
 

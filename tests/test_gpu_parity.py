@@ -3,7 +3,8 @@
 Small shapes are compared element by element for every stage; they span several query
 and key tiles, ragged frame tails (T not a multiple of B, T < B), odd query-block counts
 (a tile with one query block), sinks, no history, and k_f / k_b at or above their
-limits.  The full-size workloads (the 480p chunk the benchmark times, the large-model
+limits, and the size limits (the most frames, selected blocks and tokens per frame the
+library accepts).  The full-size workloads (the 480p chunk the benchmark times, the large-model
 stress, a rolling-cache chunk and a growth-sweep chunk) run the exact benchmark call and
 are checked on all selected indices and on sampled query blocks of the output, plus
 properties that hold at any size (every row written and finite).
@@ -41,6 +42,19 @@ SMALL = {
     "frames_1560_b128": lambda: W.random_small(9, H=2, d=128, T=1560, block=128,
                                                n_cur_frames=1, n_hist=4, n_sink=0,
                                                k_f=2, k_b=5),
+    # the size limits: n_hist + n_sink = LF_MAX_FRAMES (fused selection, 250 candidate
+    # frames, 200 kept) ...
+    "max_frames_fused": lambda: W.random_small(10, H=1, d=64, T=64, block=64,
+                                               n_cur_frames=1, n_hist=250, n_sink=6,
+                                               k_f=200, k_b=1),
+    # ... 1000 selected blocks per query block, near LF_MAX_SELECTED (the separate
+    # frame and block selection kernels; a 2016-entry key plan) ...
+    "max_selected_unfused": lambda: W.random_small(11, H=1, d=64, T=256, block=64,
+                                                   n_cur_frames=1, n_hist=252, n_sink=4,
+                                                   k_f=250, k_b=4),
+    # ... and T = LF_MAX_T tokens per frame
+    "max_T": lambda: W.random_small(12, H=1, d=64, T=16384, block=128, n_cur_frames=1,
+                                    n_hist=2, n_sink=1, k_f=2, k_b=8),
 }
 
 
