@@ -259,6 +259,22 @@ def oracle_sample(ci, budget_s=0.0, first_head=0):
     return flops, dt, torch.get_num_threads(), heads
 
 
+def oracle_single_core(ci):
+    """One head of the chunk through the oracle with torch and the BLAS pools at one
+    thread (the pools are restored afterwards).  Returns (FLOPs, seconds)."""
+    import numpy  # noqa: F401  (loads the BLAS library so its pool can be limited)
+    import torch
+    from threadpoolctl import threadpool_limits
+    n = torch.get_num_threads()
+    torch.set_num_threads(1)
+    try:
+        with threadpool_limits(limits=1):
+            f, dt, _, _ = oracle_sample(ci)
+    finally:
+        torch.set_num_threads(n)
+    return f, dt
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -573,10 +589,13 @@ def run_lf(args, rank, world, local_rank):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, dt, cores, heads = oracle_sample(ci, budget_s=10.0)
+        f1, dt1 = oracle_single_core(ci)
         line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle", "seconds": dt,
                                 "sample": f"heads 0..{heads - 1} of {sh.H} of the chunk: "
-                                          f"(a)-(d) float64 numpy, head by head"}
+                                          f"(a)-(d) float64 numpy, head by head",
+                                "single_core": {"value": f1 / dt1 / 1e12, "unit": "TFLOP/s",
+                                                "seconds": dt1, "sample": "head 0, one thread"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

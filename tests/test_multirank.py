@@ -71,3 +71,18 @@ def test_shard_heads_is_a_head_slice():
     assert torch.equal(part.q[:, 0], ci.q[:, 1])
     assert torch.equal(part.k_cache[:, :, 0], ci.k_cache[:, :, 1])
     assert part.q.is_contiguous() and part.hist_slots == ci.hist_slots
+
+
+def test_oracle_timings_are_bounded_samples():
+    """The CPU-baseline helpers: one head per sample without a budget, the torch thread
+    count restored after the single-thread run, the FLOPs those of the heads run."""
+    import lf_workloads as W
+    ci = W.tiny(0)
+    n = torch.get_num_threads()
+    f, dt, cores, heads = bench.oracle_sample(ci)
+    assert heads == 1 and f > 0 and dt > 0 and cores == n
+    f1, dt1 = bench.oracle_single_core(ci)
+    assert f1 == f and dt1 > 0
+    assert torch.get_num_threads() == n
+    f_all, _, _, heads_all = bench.oracle_sample(ci, budget_s=1e9)
+    assert heads_all == ci.shape.H and f_all == ci.shape.H * f
