@@ -11,7 +11,8 @@ the method reduces to, and invariants the method's description implies:
 * selection: exhaustive search over all k-subsets (maximal score sum, lexicographically
   smallest among equals) agrees with the top-k rule;
 * attention: with every frame and block kept, HSA is full attention, checked against
-  torch's scaled_dot_product_attention in float64; zero queries give the uniform
+  torch's scaled_dot_product_attention in float64; for arbitrary block lists it is SDPA
+  with a token mask built from the lists by another route; zero queries give the uniform
   average of the key set's values and lse = log(|key set|); probabilities are
   non-negative and sum to one; unselected keys can be permuted or replaced freely;
 * fixed complexity: the number of selected blocks does not depend on the history length;
@@ -203,6 +204,59 @@ def test_dense_equivalence_with_sdpa(T, B, F, S):
     o_ref, lse_ref = _dense_reference_sdpa(ci)
     assert np.allclose(r["O"], o_ref, rtol=0, atol=1e-12)
     assert np.allclose(r["lse"], lse_ref, rtol=0, atol=1e-12)
+
+
+def _masked_reference_sdpa(ci, block_idx):
+    """torch SDPA (float64, CPU) over current + sinks + ALL history frames with a boolean
+    token mask: a history key token (frame position f, token t) is visible to a query
+    token iff f * n_bpf + t // B is in the selected list of the query's block."""
+    sh = ci.shape
+    T, B, Fc = sh.T, sh.block, sh.n_cur_frames
+    nbpf = -(-T // B)
+    keys = [ci.k_cur.double()] + [ci.k_cache[s].double() for s in ci.sink_slots] + \
+           [ci.k_cache[s].double() for s in ci.hist_slots]
+    vals = [ci.v_cur.double()] + [ci.v_cache[s].double() for s in ci.sink_slots] + \
+           [ci.v_cache[s].double() for s in ci.hist_slots]
+    K = torch.cat(keys, 0).permute(1, 0, 2)
+    V = torch.cat(vals, 0).permute(1, 0, 2)
+    Q = ci.q.double().permute(1, 0, 2)
+    n_q, n_dense = Fc * T, Fc * T + sh.n_sink * T
+    tq = torch.arange(n_q)
+    q_block = (tq // T) * nbpf + (tq % T) // B                       # [n_q]
+    th = torch.arange(sh.n_hist * T)
+    k_block = (th // T) * nbpf + (th % T) // B                       # [F*T] global block id
+    mask = torch.ones(sh.H, n_q, n_dense + sh.n_hist * T, dtype=torch.bool)
+    for h in range(sh.H):
+        sel = torch.zeros(Fc * nbpf, sh.n_hist * nbpf, dtype=torch.bool)
+        for qb in range(Fc * nbpf):
+            sel[qb, torch.as_tensor(block_idx[h, qb], dtype=torch.long)] = True
+        mask[h, :, n_dense:] = sel[q_block][:, k_block]
+    out = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None],
+                                                           attn_mask=mask[None],
+                                                           scale=sh.scale)[0]
+    logits = torch.einsum("hqd,hkd->hqk", Q, K) * sh.scale
+    lse = torch.logsumexp(logits.masked_fill(~mask, float("-inf")), -1)
+    return out.permute(1, 0, 2).numpy(), lse.numpy()
+
+
+@pytest.mark.parametrize("seed,T,B,F,S,nsel", [(21, 100, 32, 3, 0, 5), (22, 70, 16, 4, 1, 7),
+                                               (23, 64, 64, 3, 2, 2), (24, 40, 64, 5, 0, 3)])
+def test_sparse_attention_equals_masked_sdpa(seed, T, B, F, S, nsel):
+    """Any block lists (here random, not the selection's) give the attention of a token
+    mask built from the lists: ragged last blocks, slot indirection and the joint
+    softmax over current + sinks + selected blocks are all in the mask route."""
+    nbpf = -(-T // B)
+    ci = W.random_small(seed, H=2, d=16, T=T, block=B, n_cur_frames=2, n_hist=F,
+                        n_sink=S, k_f=1, k_b=1)
+    g = np.random.default_rng(seed)
+    nqb = 2 * nbpf
+    bidx = np.stack([np.stack([np.sort(g.choice(F * nbpf, size=nsel, replace=False))
+                               for _ in range(nqb)]) for _ in range(2)])
+    o, lse = O.attention(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                         ci.hist_slots, ci.sink_slots, bidx)
+    o_ref, lse_ref = _masked_reference_sdpa(ci, bidx)
+    assert np.allclose(o, o_ref, rtol=0, atol=1e-12)
+    assert np.allclose(lse, lse_ref, rtol=0, atol=1e-12)
 
 
 def test_no_history_is_attention_over_current_and_sinks():
