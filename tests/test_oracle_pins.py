@@ -55,18 +55,22 @@ def test_block_bounds_closed_form():
     assert O.block_bounds(256, 64) == [(0, 64), (64, 128), (128, 192), (192, 256)]
 
 
-def test_pooling_ramp_closed_form():
-    T, B = 20, 8
+@pytest.mark.parametrize("T,B,blocks", [(20, 8, [(0, 8), (8, 16), (16, 20)]),   # ragged tail
+                                         (24, 8, [(0, 8), (8, 16), (16, 24)]),   # exact
+                                         (20, 32, [(0, 20)])])                   # T < B
+def test_pooling_ramp_closed_form(T, B, blocks):
     q, kc = _ramp_inputs(T, B)
     qb = O.compress_queries(q, T, B)
-    # blocks of frame f: [0,8), [8,16), [16,20) -> mean token = f*T + (s + e - 1)/2
+    nb = len(blocks)
+    # query block b of frame f covers tokens [s, e): mean token = f*T + (s + e - 1)/2
     for f in range(2):
-        for b, (s, e) in enumerate([(0, 8), (8, 16), (16, 20)]):
-            assert np.allclose(qb[:, f * 3 + b, :], f * T + (s + e - 1) / 2.0, atol=0, rtol=0)
+        for b, (s, e) in enumerate(blocks):
+            assert np.allclose(qb[:, f * nb + b, :], f * T + (s + e - 1) / 2.0, atol=0, rtol=0)
     slots = [3, 0, 4]
     kb, kf = O.compress_keys(kc, slots, T, B)
+    assert kb.shape[2] == nb
     for f, s in enumerate(slots):
-        for b, (a, e) in enumerate([(0, 8), (8, 16), (16, 20)]):
+        for b, (a, e) in enumerate(blocks):
             assert np.allclose(kb[:, f, b, :], 10.0 * s + (a + e - 1) / 8.0, rtol=0, atol=1e-12)
         assert np.allclose(kf[:, f, :], 10.0 * s + (T - 1) / 8.0, rtol=0, atol=1e-12)
 
