@@ -66,6 +66,7 @@ int check_slots(const int32_t* slots, int n, int n_slots) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? LF_OK : LF_ERR_CUDA; }
 
 constexpr size_t kMaxSmem = 227 * 1024;   // opt-in shared memory per block on sm_100
+static_assert(LF_MAX_PLAN == lf::kMaxPlan, "the header's key-plan limit is the kernels'");
 
 // --------------------------------------------------------------- tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;

@@ -74,6 +74,8 @@ extern "C" {
 #define LF_MAX_FRAMES       256     /* n_sink + n_hist                                  */
 #define LF_MAX_T            16384   /* tokens per frame                                 */
 #define LF_MAX_SELECTED     1024    /* kf * kb per query block                          */
+#define LF_MAX_PLAN         2048    /* key blocks per 128-row query tile:
+                                       n_sink * n_bpf + (block == 64 ? 2 : 1) * kf * kb  */
 
 typedef struct lf_shape {
     int32_t H;                /* heads, >= 1                                              */

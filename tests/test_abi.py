@@ -58,6 +58,11 @@ def _attn(lib, shape, hist=(0, 1, 2, 3), sinks=(), ws=1 << 20, wsptr=FAKE, bidx=
     (dict(n_cur_frames=0), 1), (dict(T=0), 1), (dict(T=20000), 2), (dict(n_hist=-1), 1),
     (dict(k_f=0), 1), (dict(k_b=0), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
     (dict(n_hist=300, n_slots=300), 2),
+    # one past each size limit of the header
+    (dict(T=16385), 2),                                                    # LF_MAX_T
+    (dict(n_hist=250, n_sink=7, n_slots=257, k_f=1), 2),                   # LF_MAX_FRAMES
+    (dict(T=1600, n_hist=41, n_slots=41, k_f=41, k_b=25), 2),              # LF_MAX_SELECTED
+    (dict(T=1600, n_hist=40, n_sink=4, n_slots=44, k_f=40, k_b=25), 2),    # LF_MAX_PLAN
 ])
 def test_shape_validation(lib, kw, code):
     assert _attn(lib, _shape(**kw), hist=tuple(range(min(kw.get("n_hist", 4), 256)))
