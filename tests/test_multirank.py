@@ -86,3 +86,20 @@ def test_oracle_timings_are_bounded_samples():
     assert torch.get_num_threads() == n
     f_all, _, _, heads_all = bench.oracle_sample(ci, budget_s=1e9)
     assert heads_all == ci.shape.H and f_all == ci.shape.H * f
+
+
+def test_clock_summary_from_fake_rows():
+    """The clock record of the JSON line from nvidia-smi rows (a fake of its CSV output):
+    median SM clock, max clock, the active throttle reasons; bad rows are skipped."""
+    row = "0, {sm}, 1965, 700.5, 0x{m}, {hw}, Not Active, Not Active, {pc}"
+    rows = [row.format(sm=1965, m="0", hw="Not Active", pc="Not Active"),
+            row.format(sm=1800, m="4", hw="Not Active", pc="Active"),
+            row.format(sm=1900, m="4", hw="Not Active", pc="Active"),
+            "0, [N/A], 1965, 700, 0x0, Not Active, Not Active, Not Active, Not Active",
+            "garbage"]
+    out = bench.summarise_clocks(rows)
+    assert out == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3}
+    rows.append(row.format(sm=1200, m="8", hw="Active", pc="Not Active"))
+    assert bench.summarise_clocks(rows)["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert bench.summarise_clocks([])["sm_mhz"] is None
