@@ -36,7 +36,6 @@ All arithmetic is float64 on values upcast from the bf16 inputs.
 """
 from __future__ import annotations
 
-import itertools
 import math
 from typing import List, Sequence, Tuple
 
@@ -46,7 +45,7 @@ __all__ = [
     "block_bounds", "n_blocks", "compress_queries", "compress_keys", "frame_scores",
     "topk_lower_index", "select_frames", "block_scores_in_frame", "select_blocks",
     "key_set", "attention_qblock", "attention", "forward_chunk", "boundary_gap",
-    "executed_flops", "selection_bytes",
+    "select_blocks_1d", "executed_flops",
 ]
 
 
@@ -293,7 +292,3 @@ def executed_flops(shape, block_idx) -> int:
             total += (e - s) * (dense_keys + nsel)
     return 4 * shape.d * total
 
-
-def selection_bytes(shape) -> int:
-    """HBM bytes the compression must read: the current queries and the history keys."""
-    return 2 * shape.H * shape.d * shape.T * (shape.n_cur_frames + shape.n_hist)
