@@ -98,23 +98,18 @@ def attn_sources_sha256() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary of this workload,
-    or None if there is none or the kernel's sources changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}.md")
+    """DRAM bytes per attention launch from the committed ncu figures of this workload
+    (profiles/attn_kernel_<workload>.json), or None if there are none or the kernel's
+    sources changed since they were taken."""
+    path = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}.json")
     if not os.path.exists(path):
         return None
-    vals = {}
     with open(path) as f:
-        for line in f:
-            if ":" in line and line.startswith("- "):
-                k, v = line[2:].split(":", 1)
-                vals[k.strip()] = v.strip().strip("`")
+        vals = json.load(f)
     if vals.get("source_sha256") != attn_sources_sha256():
         return None
-    try:
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    v = vals.get("dram_bytes_per_launch")
+    return float(v) if v is not None else None
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -230,44 +225,73 @@ def summarise_clocks(rows):
             "reasons": sorted(reasons), "samples": len(sm)}
 
 
+CONFIG_NAMES = ("480p", "large", "rolling", "growth")
+
+
 def make_workload(name, seed):
+    """(chunks, description) of a benchmark workload.  A step processes every chunk of the
+    list once: the 480p and large chunks alone, the rolling cache's steady-state chunk (3
+    sink frames + the last 21 frames), or the 7 chunks of the growth sweep, whose (k_f,
+    k_b) budgets come from the library's growth schedule (lf_cag_schedule)."""
     import lf_workloads as W
     if name == "480p":
-        return W.p480(seed), "Self-Forcing-shaped 480p chunk: H=12 d=128 T=1560 (30x52), " \
-                             "chunk 3 frames (4680 queries), 18 history frames, B=64, k_f=6, k_b=12"
+        return [W.p480(seed)], "Self-Forcing-shaped 480p chunk: H=12 d=128 T=1560 (30x52), " \
+                               "chunk 3 frames (4680 queries), 18 history frames, B=64, k_f=6, k_b=12"
     if name == "large":
-        return W.large(seed), "large-model stress: H=40 d=128 T=1560, chunk 3, " \
-                              "42 history frames, B=128, k_f=8, k_b=5"
-    raise SystemExit(f"unknown config {name}")
+        return [W.large(seed)], "large-model stress: H=40 d=128 T=1560, chunk 3, " \
+                                "42 history frames, B=128, k_f=8, k_b=5"
+    if name == "rolling":
+        ci = None
+        for ci in W.rolling(seed, n_chunks=9):
+            pass
+        return [ci], "rolling-cache steady state (chunk 9 of the 60-frame generation): H=12 " \
+                     "d=128 T=1560, chunk 3 frames, 3 sink frames + 21 rolling history frames, " \
+                     "B=64, k_f=4, k_b=6"
+    if name == "growth":
+        import block_sparse_attention_46_b200 as lf
+        chunks = W.growth_sweep(seed)
+        nbpf = -(-chunks[0].shape.T // chunks[0].shape.block)
+        keep, kf, kb = lf.lf_cag_schedule(7, 2, 0.8, 0.9, [c.shape.n_hist for c in chunks],
+                                          nbpf, 6)
+        for c, f, b in zip(chunks, kf, kb):
+            if c.shape.n_hist > 0 and (c.shape.k_f, c.shape.k_b) != (f, b):
+                raise SystemExit(f"growth budget {(c.shape.k_f, c.shape.k_b)} != schedule {(f, b)}")
+        return chunks, "chunk-aware growth sweep: 7 chunks of 3 frames at the 480p shape " \
+                       "(H=12 d=128 T=1560, B=64), history 0,3,...,18 frames, keep ratio " \
+                       "1 then mean 0.2 over chunks 2-7 (k_f, k_b from lf_cag_schedule: " + \
+                       ", ".join(f"({a},{b})" for a, b in zip(kf, kb)) + ")"
+    raise SystemExit(f"unknown config {name} (one of {', '.join(CONFIG_NAMES)})")
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_sample(ci, budget_s=0.0, first_head=0):
-    """Runs the float64 oracle (a)-(d) head by head (each head is an independent problem)
-    until `budget_s` seconds are spent (at least one head): a bounded sample of the chunk.
-    Returns (executed FLOPs of the sample, seconds, cores, heads run)."""
+def oracle_sample(chunks, budget_s=0.0, first=0):
+    """Runs the float64 oracle (a)-(d) one (chunk, head) at a time (each head of a chunk is
+    an independent problem), starting at unit `first`, until `budget_s` seconds are spent
+    (at least one unit): a bounded sample of the workload.  Returns (executed FLOPs of the
+    sample, seconds, cores, units run)."""
     from dataclasses import replace
     from oracle import hsa64 as O
     import torch
-    sh = ci.shape
-    s1 = replace(sh, H=1)
-    flops, dt, heads = 0, 0.0, 0
-    for i in range(sh.H):
-        h = (first_head + i) % sh.H
+    units = [(c, h) for c in range(len(chunks)) for h in range(chunks[c].shape.H)]
+    flops, dt, n = 0, 0.0, 0
+    for i in range(len(units)):
+        c, h = units[(first + i) % len(units)]
+        ci = chunks[c]
+        s1 = replace(ci.shape, H=1)
         sl = lambda t: t[..., h:h + 1, :].contiguous()
         t0 = time.perf_counter()
         r = O.forward_chunk(s1, sl(ci.q), sl(ci.k_cur), sl(ci.v_cur), sl(ci.k_cache),
                             sl(ci.v_cache), ci.hist_slots, ci.sink_slots)
         dt += time.perf_counter() - t0
         flops += executed_flops(s1, r.get("block_idx"))
-        heads += 1
+        n += 1
         if dt >= budget_s:
             break
-    return flops, dt, torch.get_num_threads(), heads
+    return flops, dt, torch.get_num_threads(), n
 
 
-def oracle_single_core(ci):
-    """One head of the chunk through the oracle with torch and the BLAS pools at one
+def oracle_single_core(chunks):
+    """One head of the workload through the oracle with torch and the BLAS pools at one
     thread (the pools are restored afterwards).  Returns (FLOPs, seconds)."""
     import numpy  # noqa: F401  (loads the BLAS library so its pool can be limited)
     import torch
@@ -276,7 +300,7 @@ def oracle_single_core(ci):
     torch.set_num_threads(1)
     try:
         with threadpool_limits(limits=1):
-            f, dt, _, _ = oracle_sample(ci)
+            f, dt, _, _ = oracle_sample(chunks[-1:])
     finally:
         torch.set_num_threads(n)
     return f, dt
@@ -285,16 +309,16 @@ def oracle_single_core(ci):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    ci, desc = make_workload(args.config, 0)
+    chunks, desc = make_workload(args.config, 0)
     for _ in range(min(args.warmup, 1)):
-        oracle_sample(ci)
+        oracle_sample(chunks)
     tot_f, tot_t, cores = 0, 0.0, 1
     for k in range(args.steps):
-        f, t, cores, _ = oracle_sample(ci, first_head=k)
+        f, t, cores, _ = oracle_sample(chunks, first=k)
         tot_f += f
         tot_t += t
     value = tot_f / tot_t / 1e12
-    sample = f"one head of the {args.config} chunk per step ((a)-(d), float64 numpy)"
+    sample = f"one (chunk, head) of the {args.config} workload per step ((a)-(d), float64 numpy)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -313,6 +337,53 @@ METRIC = "ms/chunk & effective TFLOP/s, hierarchical sparse attn, 480p chunk sha
 
 
 # ----------------------------------------------------------------------------- GPU arm
+class ChunkRun:
+    """Device tensors and C-ABI calls of one chunk of a workload."""
+
+    def __init__(self, lf, ci, dev):
+        import torch
+        self.lf, self.ci, self.sh = lf, ci, ci.shape
+        sh = self.sh
+        nbpf, nqb, kf, kb = lf.derived(sh)
+        self.t = {k: getattr(ci, k).to(dev) for k in ("q", "k_cur", "v_cur", "k_cache", "v_cache")}
+        self.bidx = torch.empty(sh.H, nqb, max(kf * kb, 1), dtype=torch.int32, device=dev)
+        self.sws = torch.empty(max(lf.lf_select_workspace_size(sh), 256), dtype=torch.uint8,
+                               device=dev)
+        self.out = torch.empty_like(self.t["q"])
+        self.lse = torch.empty(sh.H, self.t["q"].shape[0], device=dev)
+        self.ws = torch.empty(max(lf.lf_attn_workspace_size(sh), 256), dtype=torch.uint8,
+                              device=dev)
+
+    def select(self):
+        if self.sh.n_hist > 0:
+            t = self.t
+            self.lf.lf_select_chunk(self.sh, t["q"], t["k_cache"], self.ci.hist_slots, self.bidx,
+                                    self.sws)
+
+    def attend(self):
+        t = self.t
+        self.lf.lf_block_sparse_attn(self.sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"],
+                                     t["v_cache"], self.ci.hist_slots, self.ci.sink_slots,
+                                     self.bidx, self.out, self.lse, self.ws)
+
+    def launches(self) -> int:
+        # selection kernels | plan, schedule, attn (+ merge)
+        return selection_launches(self.sh) + 3 + (1 if tail_split(self.sh) else 0)
+
+
+def capture(fn, stream, cap):
+    """fn() captured once into a CUDA graph on the side stream `cap`."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    return g
+
+
 def run_lf(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -321,23 +392,19 @@ def run_lf(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     lf.load()
     if args.shard == "heads":
-        # one chunk split by heads over the ranks (strong scaling): same seed everywhere
-        ci, desc = make_workload(args.config, 0)
-        h0, h1 = head_shard(ci.shape.H, world, rank)
-        if h1 <= h0:
-            raise SystemExit(f"--shard heads needs at most H={ci.shape.H} ranks")
-        ci = shard_heads(ci, h0, h1)
+        # one workload split by heads over the ranks (strong scaling): same seed everywhere
+        chunks, desc = make_workload(args.config, 0)
+        split = []
+        for ci in chunks:
+            h0, h1 = head_shard(ci.shape.H, world, rank)
+            if h1 <= h0:
+                raise SystemExit(f"--shard heads needs at most H={ci.shape.H} ranks")
+            split.append(shard_heads(ci, h0, h1))
+        chunks = split
         desc += f"; heads split over {world} ranks"
     else:
-        ci, desc = make_workload(args.config, rank)
-    sh = ci.shape
-    nbpf, nqb, kf, kb = lf.derived(sh)
-    t = {k: getattr(ci, k).to(dev) for k in ("q", "k_cur", "v_cur", "k_cache", "v_cache")}
-    bidx = torch.empty(sh.H, nqb, max(kf * kb, 1), dtype=torch.int32, device=dev)
-    sws = torch.empty(lf.lf_select_workspace_size(sh), dtype=torch.uint8, device=dev)
-    out = torch.empty_like(t["q"])
-    lse = torch.empty(sh.H, t["q"].shape[0], device=dev)
-    ws = torch.empty(max(lf.lf_attn_workspace_size(sh), 256), dtype=torch.uint8, device=dev)
+        chunks, desc = make_workload(args.config, rank)
+    runs = [ChunkRun(lf, ci, dev) for ci in chunks]
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     flush_sink = torch.empty((), dtype=torch.int64, device=dev)
 
@@ -350,12 +417,12 @@ def run_lf(args, rank, world, local_rank):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
     def sel_stage():
-        if sh.n_hist > 0:
-            lf.lf_select_chunk(sh, t["q"], t["k_cache"], ci.hist_slots, bidx, sws)
+        for r in runs:
+            r.select()
 
     def att_stage():
-        lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
-                                ci.hist_slots, ci.sink_slots, bidx, out, lse, ws)
+        for r in runs:
+            r.attend()
 
     # warm up eagerly, then capture each stage in a CUDA graph (removes host overhead
     # between launches; the graphs replay exactly the kernels of the C-ABI calls)
@@ -363,16 +430,8 @@ def run_lf(args, rank, world, local_rank):
         sel_stage()
         att_stage()
     torch.cuda.synchronize()
-    g_sel, g_att = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream()
-    cap.wait_stream(stream)
-    with torch.cuda.stream(cap):
-        with torch.cuda.graph(g_sel, stream=cap):
-            sel_stage()
-        with torch.cuda.graph(g_att, stream=cap):
-            att_stage()
-    stream.wait_stream(cap)
-    torch.cuda.synchronize()
+    g_sel, g_att = capture(sel_stage, stream, cap), capture(att_stage, stream, cap)
 
     def step(record=False):
         if record:
@@ -388,9 +447,9 @@ def run_lf(args, rank, world, local_rank):
         flush_l2()
         step()
     torch.cuda.synchronize()
-    flops = executed_flops(sh, bidx.cpu().numpy())
-    # selection kernels | plan, schedule, attn (+ merge)
-    launches_per_step = selection_launches(sh) + 3 + (1 if tail_split(sh) else 0)
+    flops = sum(executed_flops(r.sh, r.bidx.cpu().numpy()) for r in runs)
+    sel_bytes = sum(selection_bytes(r.sh) for r in runs if r.sh.n_hist > 0)
+    launches_per_step = sum(r.launches() for r in runs)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -422,189 +481,208 @@ def run_lf(args, rank, world, local_rank):
         job_flops = float(world * flops)
         value = weak_scaling_value(flops, world, ms_step)
 
-    # incremental compression: history block means kept per cache slot; per step the frames
-    # that enter the cache (three slots re-pooled here, their keys unchanged, so the
-    # selection is the same) are pooled and the selection reads the pooled-key cache
-    inc = None
-    if sh.n_hist > 0:
-        k_pool = torch.empty(lf.lf_pooled_cache_bytes(sh) // 4, dtype=torch.float32, device=dev)
-        lf.lf_pool_frames(sh, t["k_cache"], sorted(set(ci.hist_slots)), k_pool)
-        new_slots = list(ci.hist_slots[:sh.n_cur_frames])
-        bidx_c = torch.empty_like(bidx)
-
-        def sel_cached():
-            lf.lf_pool_frames(sh, t["k_cache"], new_slots, k_pool)
-            lf.lf_select_chunk_cached(sh, t["q"], k_pool, ci.hist_slots, bidx_c, sws)
-        for _ in range(3):
-            sel_cached()
-        torch.cuda.synchronize()
-        g_selc = torch.cuda.CUDAGraph()
-        cap.wait_stream(stream)
-        with torch.cuda.stream(cap):
-            with torch.cuda.graph(g_selc, stream=cap):
-                sel_cached()
-        stream.wait_stream(cap)
-        torch.cuda.synchronize()
-        n_inc = max(3, min(args.steps, 200))
-        selc_ms, attc_ms = [], []
-        for _ in range(n_inc):
-            flush_l2()
-            ev[0].record(stream)
-            g_selc.replay()
-            ev[1].record(stream)
-            g_att.replay()
-            ev[2].record(stream)
-            ev[2].synchronize()
-            selc_ms.append(ev[0].elapsed_time(ev[1]))
-            attc_ms.append(ev[1].elapsed_time(ev[2]))
-        same = bool(torch.equal(bidx_c, bidx))
-        inc_bytes = 2 * sh.H * sh.d * sh.T * (2 * sh.n_cur_frames)      # Q + the new frames' K
-        selc_mean = max_over_ranks(statistics.mean(selc_ms), dev)
-        inc = {"ms_selection_abc": selc_mean,
-               "ms_per_step": selc_mean + max_over_ranks(statistics.mean(attc_ms), dev),
-               "selection_mb_per_chunk": inc_bytes / 1e6,
-               "selection_gbs": inc_bytes / (selc_mean * 1e-3) / 1e9,
-               "indices_equal_full_recompute": same,
-               "api": "lf_pool_frames (the chunk's frames entering the cache) + "
-                      "lf_select_chunk_cached, then lf_block_sparse_attn"}
-
-    # the one-dimensional ablation (no frame stage): its selection and the attention over
-    # the blocks it selects (the same number per query block, not clustered by frame)
-    abl = None
-    if sh.n_hist > 0 and sh.n_hist * -(-sh.T // sh.block) <= 2048:
-        bidx_1d = torch.empty_like(bidx)
-        out_1d = torch.empty_like(out)
-        ws_1d = torch.empty_like(ws)
-
-        def stages_1d():
-            lf.lf_select_chunk_1d(sh, t["q"], t["k_cache"], ci.hist_slots, bidx_1d, sws)
-            lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"],
-                                    t["v_cache"], ci.hist_slots, ci.sink_slots, bidx_1d,
-                                    out_1d, None, ws_1d)
-        for _ in range(3):
-            stages_1d()
-        torch.cuda.synchronize()
-        g_1d = torch.cuda.CUDAGraph()
-        cap.wait_stream(stream)
-        with torch.cuda.stream(cap):
-            with torch.cuda.graph(g_1d, stream=cap):
-                stages_1d()
-        stream.wait_stream(cap)
-        torch.cuda.synchronize()
-        ms_1d = []
-        for _ in range(max(3, min(args.steps, 200))):
-            flush_l2()
-            ev[0].record(stream)
-            g_1d.replay()
-            ev[1].record(stream)
-            ev[1].synchronize()
-            ms_1d.append(ev[0].elapsed_time(ev[1]))
-        f1d = executed_flops(sh, bidx_1d.cpu().numpy())
-        m1d = max_over_ranks(statistics.mean(ms_1d), dev)
-        abl = {"ms_per_step": m1d, "executed_gflop_per_chunk": f1d / 1e9,
-               "tflops": f1d / (m1d * 1e-3) / 1e12,
-               "api": "lf_select_chunk_1d + lf_block_sparse_attn"}
-
-    # e2e through lf_forward_chunk with host buffers: every step copies its chunk's Q, K, V
-    # from pinned host memory, runs the call, and copies the output back.  Two chunks are
-    # in flight: uploads, compute and downloads run on three streams (separate copy
-    # engines), with double-buffered device inputs/outputs.
-    hq = {k: t[k].cpu().pin_memory() for k in ("q", "k_cur", "v_cur")}
-    dq = [{k: torch.empty_like(t[k]) for k in hq} for _ in range(2)]
-    dout = [torch.empty_like(out) for _ in range(2)]
-    hout = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
-    fws = torch.empty(lf.lf_forward_workspace_size(sh), dtype=torch.uint8, device=dev)
-    n_e2e = max(4, min(args.steps, 50))
-    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def e2e_run(n):
-        for i in range(n):
-            b = i % 2
-            if i >= 2:
-                s_in.wait_event(ev_comp[b])          # step i-2 has consumed these inputs
-            with torch.cuda.stream(s_in):
-                for k in hq:
-                    dq[b][k].copy_(hq[k], non_blocking=True)
-            ev_in[b].record(s_in)
-            s_comp.wait_event(ev_in[b])
-            if i >= 2:
-                s_comp.wait_event(ev_out[b])         # step i-2's output has been read back
-            lf.lf_forward_chunk(sh, dq[b]["q"], dq[b]["k_cur"], dq[b]["v_cur"], t["k_cache"],
-                                t["v_cache"], ci.hist_slots, ci.sink_slots, dout[b], None, None,
-                                fws, stream=s_comp)
-            ev_comp[b].record(s_comp)
-            s_out.wait_event(ev_comp[b])
-            with torch.cuda.stream(s_out):
-                hout[b].copy_(dout[b], non_blocking=True)
-            ev_out[b].record(s_out)
-
-    e2e_run(4)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    s_in.wait_stream(stream)
-    e0.record(s_in)
-    e2e_run(n_e2e)
-    s_out.wait_stream(s_in)
-    s_out.wait_stream(s_comp)
-    e1.record(s_out)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
-    e2e_same = bool(torch.equal(hout[(n_e2e - 1) % 2], out.cpu()))
-    h2d = sum(hq[k].numel() * hq[k].element_size() for k in hq)
-    d2h = hout[0].numel() * hout[0].element_size()
+    single = len(runs) == 1 and runs[0].sh.n_hist > 0
+    inc = incremental_compression(lf, runs[0], args, stream, cap, ev, flush_l2, g_att) \
+        if single else None
+    abl = ablation_1d(lf, runs[0], args, stream, cap, ev, flush_l2) if single else None
+    e2e = end_to_end(lf, runs, args, stream, dev, world, job_flops)
 
     pk, src = peaks()
     att_mean = statistics.mean(att_ms)
     sel_mean = statistics.mean(sel_ms)
     att_tflops = flops / (att_mean * 1e-3) / 1e12
-    sel_gbs = selection_bytes(sh) / (sel_mean * 1e-3) / 1e9
+    n_chunks = len(runs)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; per-frame key centroids, planted related frames)",
-        "config": {"workload": desc,
+        "config": {"workload": desc, "chunks_per_step": n_chunks,
                    "l2": "flushed before every timed step (256 MB written, then read back)",
-                   "executed_gflop_per_chunk": flops / 1e9,
-                   "selection_mb_per_chunk": selection_bytes(sh) / 1e6,
+                   "executed_gflop_per_step": flops / 1e9,
+                   "selection_mb_per_step": sel_bytes / 1e6,
+                   "ms_per_chunk": ms_step / n_chunks,
                    "ms_selection_abc": sel_mean, "ms_attention_d": att_mean,
                    "selection_share": sel_mean / (sel_mean + att_mean)},
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": att_tflops / pk["bf16_tflops"],
-                     "traffic": profiled_traffic(args.config),
+                     "traffic": profiled_traffic(args.config) if n_chunks == 1 else None,
                      "kernel": "stage (d): plan + schedule + attn_kernel + merge (lf_block_sparse_attn)",
                      "peak_source": f"{src} bf16_tflops (burst)"},
-        "roofline_selection": {"bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"],
-                               "unit": "GB/s", "frac": sel_gbs / pk["hbm_gbs"],
-                               "kernels": "pool_blocks + block_scores + select_pick (lf_select_chunk)",
-                               "peak_source": f"{src} hbm_gbs"},
-        "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "lf_forward_chunk per step, two chunks in flight (uploads, compute and "
-                       "downloads on three streams)",
-                "output_equals_device_path": e2e_same},
+        "e2e": e2e,
         "incremental_compression": inc,
         "ablation_1d": abl,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if sel_bytes > 0:
+        sel_gbs = sel_bytes / (sel_mean * 1e-3) / 1e9
+        line["roofline_selection"] = {
+            "bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": sel_gbs / pk["hbm_gbs"],
+            "kernels": "pool_blocks + block_scores + select_pick (lf_select_chunk)",
+            "peak_source": f"{src} hbm_gbs"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, dt, cores, heads = oracle_sample(ci, budget_s=10.0)
-        f1, dt1 = oracle_single_core(ci)
+        f, dt, cores, n = oracle_sample(chunks, budget_s=10.0)
+        f1, dt1 = oracle_single_core(chunks)
         line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle", "seconds": dt,
-                                "sample": f"heads 0..{heads - 1} of {sh.H} of the chunk: "
+                                "sample": f"{n} (chunk, head) units of the workload in order: "
                                           f"(a)-(d) float64 numpy, head by head",
                                 "single_core": {"value": f1 / dt1 / 1e12, "unit": "TFLOP/s",
-                                                "seconds": dt1, "sample": "head 0, one thread"}}
+                                                "seconds": dt1,
+                                                "sample": "head 0 of the last chunk, one thread"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def incremental_compression(lf, r, args, stream, cap, ev, flush_l2, g_att):
+    """History block means kept per cache slot (the pooled-key cache): per step the frames
+    that enter the cache (three slots re-pooled here, their keys unchanged, so the
+    selection is the same) are pooled and the selection reads the pooled-key cache."""
+    import torch
+    sh, t, ci = r.sh, r.t, r.ci
+    dev = t["q"].device
+    k_pool = torch.empty(lf.lf_pooled_cache_bytes(sh) // 4, dtype=torch.float32, device=dev)
+    lf.lf_pool_frames(sh, t["k_cache"], sorted(set(ci.hist_slots)), k_pool)
+    new_slots = list(ci.hist_slots[:sh.n_cur_frames])
+    bidx_c = torch.empty_like(r.bidx)
+
+    def sel_cached():
+        lf.lf_pool_frames(sh, t["k_cache"], new_slots, k_pool)
+        lf.lf_select_chunk_cached(sh, t["q"], k_pool, ci.hist_slots, bidx_c, r.sws)
+    for _ in range(3):
+        sel_cached()
+    torch.cuda.synchronize()
+    g_selc = capture(sel_cached, stream, cap)
+    selc_ms, attc_ms = [], []
+    for _ in range(max(3, min(args.steps, 200))):
+        flush_l2()
+        ev[0].record(stream)
+        g_selc.replay()
+        ev[1].record(stream)
+        g_att.replay()
+        ev[2].record(stream)
+        ev[2].synchronize()
+        selc_ms.append(ev[0].elapsed_time(ev[1]))
+        attc_ms.append(ev[1].elapsed_time(ev[2]))
+    same = bool(torch.equal(bidx_c, r.bidx))
+    inc_bytes = 2 * sh.H * sh.d * sh.T * (2 * sh.n_cur_frames)      # Q + the new frames' K
+    selc_mean = max_over_ranks(statistics.mean(selc_ms), dev)
+    return {"ms_selection_abc": selc_mean,
+            "ms_per_step": selc_mean + max_over_ranks(statistics.mean(attc_ms), dev),
+            "selection_mb_per_chunk": inc_bytes / 1e6,
+            "selection_gbs": inc_bytes / (selc_mean * 1e-3) / 1e9,
+            "indices_equal_full_recompute": same,
+            "api": "lf_pool_frames (the chunk's frames entering the cache) + "
+                   "lf_select_chunk_cached, then lf_block_sparse_attn"}
+
+
+def ablation_1d(lf, r, args, stream, cap, ev, flush_l2):
+    """The one-dimensional ablation (no frame stage): its selection and the attention over
+    the blocks it selects (the same number per query block, not clustered by frame)."""
+    import torch
+    sh, t, ci = r.sh, r.t, r.ci
+    if sh.n_hist * -(-sh.T // sh.block) > 2048:
+        return None
+    dev = t["q"].device
+    bidx_1d = torch.empty_like(r.bidx)
+    out_1d = torch.empty_like(r.out)
+    ws_1d = torch.empty_like(r.ws)
+
+    def stages_1d():
+        lf.lf_select_chunk_1d(sh, t["q"], t["k_cache"], ci.hist_slots, bidx_1d, r.sws)
+        lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"],
+                                t["v_cache"], ci.hist_slots, ci.sink_slots, bidx_1d,
+                                out_1d, None, ws_1d)
+    for _ in range(3):
+        stages_1d()
+    torch.cuda.synchronize()
+    g_1d = capture(stages_1d, stream, cap)
+    ms_1d = []
+    for _ in range(max(3, min(args.steps, 200))):
+        flush_l2()
+        ev[0].record(stream)
+        g_1d.replay()
+        ev[1].record(stream)
+        ev[1].synchronize()
+        ms_1d.append(ev[0].elapsed_time(ev[1]))
+    f1d = executed_flops(sh, bidx_1d.cpu().numpy())
+    m1d = max_over_ranks(statistics.mean(ms_1d), dev)
+    return {"ms_per_step": m1d, "executed_gflop_per_chunk": f1d / 1e9,
+            "tflops": f1d / (m1d * 1e-3) / 1e12,
+            "api": "lf_select_chunk_1d + lf_block_sparse_attn"}
+
+
+def end_to_end(lf, runs, args, stream, dev, world, job_flops):
+    """The metric through lf_forward_chunk with host buffers: every chunk of every step
+    copies its Q, K, V from pinned host memory, runs the call, and copies the output back.
+    Two chunks are in flight: uploads, compute and downloads run on three streams
+    (separate copy engines), with double-buffered device inputs/outputs; the KV cache is
+    model state and stays resident."""
+    import torch
+    n = len(runs)
+    hq = [{k: r.t[k].cpu().pin_memory() for k in ("q", "k_cur", "v_cur")} for r in runs]
+    dq = [{k: torch.empty_like(runs[0].t[k]) for k in ("q", "k_cur", "v_cur")} for _ in range(2)]
+    dout = [torch.empty_like(runs[0].out) for _ in range(2)]
+    hout = [torch.empty(runs[0].out.shape, dtype=runs[0].out.dtype, pin_memory=True)
+            for _ in range(2)]
+    fws = torch.empty(max(lf.lf_forward_workspace_size(r.sh) for r in runs), dtype=torch.uint8,
+                      device=dev)
+    steps = max(4, min(args.steps, 50 // n if n > 1 else 50))
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for r in runs:
+        assert r.t["q"].shape == runs[0].t["q"].shape    # one buffer shape serves every chunk
+
+    def run(n_steps):
+        for i in range(n_steps * n):
+            b, c = i % 2, i % n
+            r = runs[c]
+            if i >= 2:
+                s_in.wait_event(ev_comp[b])          # chunk i-2 has consumed these inputs
+            with torch.cuda.stream(s_in):
+                for k in hq[c]:
+                    dq[b][k].copy_(hq[c][k], non_blocking=True)
+            ev_in[b].record(s_in)
+            s_comp.wait_event(ev_in[b])
+            if i >= 2:
+                s_comp.wait_event(ev_out[b])         # chunk i-2's output has been read back
+            lf.lf_forward_chunk(r.sh, dq[b]["q"], dq[b]["k_cur"], dq[b]["v_cur"],
+                                r.t["k_cache"], r.t["v_cache"], r.ci.hist_slots,
+                                r.ci.sink_slots, dout[b], None, None, fws, stream=s_comp)
+            ev_comp[b].record(s_comp)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                hout[b].copy_(dout[b], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    run(1)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    s_in.wait_stream(stream)
+    e0.record(s_in)
+    run(steps)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_comp)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+    last = (steps * n - 1)
+    same = bool(torch.equal(hout[last % 2], runs[last % n].out.cpu()))
+    h2d = sum(sum(x.numel() * x.element_size() for x in h.values()) for h in hq)
+    d2h = n * hout[0].numel() * hout[0].element_size()
+    return {"value": job_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "lf_forward_chunk per chunk, two chunks in flight (uploads, compute and "
+                   "downloads on three streams)",
+            "output_equals_device_path": same}
 
 
 def main():
@@ -613,7 +691,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lf", choices=["lf", "reference"])
-    ap.add_argument("--config", default="480p")
+    ap.add_argument("--config", default="480p", choices=CONFIG_NAMES)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shard", default="chunks", choices=["chunks", "heads"],
                     help="chunks: one chunk per rank (weak scaling); heads: one chunk split "

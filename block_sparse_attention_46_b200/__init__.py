@@ -21,7 +21,7 @@ __all__ = [
     "lf_select_chunk", "lf_select_workspace_size", "lf_block_sparse_attn_noalloc",
     "lf_noalloc_scratch_bytes", "lf_pooled_cache_bytes", "lf_pool_frames",
     "lf_select_chunk_cached", "lf_cag_schedule", "lf_select_chunk_1d",
-    "lf_status_string", "lf_abi_version", "derived", "LIB_PATH",
+    "lf_status_string", "lf_abi_version", "lf_debug_configure", "derived", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblf.so")
@@ -64,8 +64,8 @@ _SIGS = {
     "lf_device_status": (ctypes.c_int, [ctypes.c_int]),
     "lf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "lf_abi_version": (ctypes.c_int, []),
-    "lf_debug_exp2_poly": (ctypes.c_int, [_P, _P, ctypes.c_int, _P]),
     "lf_noalloc_scratch_bytes": (_SZ, []),
+    "lf_debug_configure": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int, ctypes.c_int]),
     "lf_pooled_cache_bytes": (_SZ, [_SHP]),
     "lf_cag_schedule": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                        ctypes.c_float, _I32P, ctypes.c_int32, ctypes.c_int32,
@@ -144,10 +144,11 @@ def lf_device_status(reset: bool = True) -> int:
     return load().lf_device_status(1 if reset else 0)
 
 
-def lf_debug_exp2_poly(x, y, stream=None):
-    """Test hook: the attention softmax's FMA-pipe exponential, y = 2^x (x <= 0)."""
-    _check(load().lf_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
-           "lf_debug_exp2_poly")
+def lf_debug_configure(wait_limit_ns: int = 0, stall: bool = False, tail_split: bool = True):
+    """Test hook: wait limit of the device waits, a stalled first CTA, and whether the last
+    partial wave of query tiles may be split (defaults restored by calling it with none)."""
+    _check(load().lf_debug_configure(int(wait_limit_ns), 1 if stall else 0,
+                                     1 if tail_split else 0), "lf_debug_configure")
 
 
 def lf_compress(shape, q, k_cache, hist_slots, q_blk, k_blk, k_frm, stream=None):

@@ -176,14 +176,17 @@ struct Split {
   int n_whole, n_tail, pieces;
 };
 
+// Test hooks set by lf_debug_configure (process-wide; defaults: 2 s wait limit, no stall,
+// tail split allowed).
+uint64_t g_dbg_wait_limit_ns = lf::kWaitLimitNs;
+int g_dbg_stall = 0;
+int g_dbg_tail_split = 1;
+
 Split make_split(const Dims& D, int n_sm) {
   const int ntot = lf::tile_count(D) * D.H;
   Split sp{ntot, 0, 1};
-  if (n_sm <= 0) return sp;
+  if (n_sm <= 0 || !g_dbg_tail_split) return sp;
   const int R = ntot % n_sm;
-#ifdef LF_NO_TAIL_SPLIT
-  return sp;
-#endif
   if (R == 0 || 2 * R > n_sm) return sp;
   int p = n_sm / R;
   p = p < lf::kMaxPieces ? p : lf::kMaxPieces;
@@ -278,6 +281,8 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   p.pieces = sp.pieces;
   p.part_o = w.part_o;
   p.part_ml = w.part_ml;
+  p.wait_limit_ns = g_dbg_wait_limit_ns;
+  p.debug_stall = g_dbg_stall;
   for (int i = 0; i < D.S; ++i) p.slots[i] = sink_slots[i];
   for (int i = 0; i < D.F; ++i) p.slots[D.S + i] = hist_slots[i];
   const int grid = sp.n_whole + sp.n_tail * sp.pieces;
@@ -374,29 +379,61 @@ int run_select(const Dims& D, const void* q, const void* k_cache, const int32_t*
 }
 
 // ---------------------------------------------------------------- fixed scratch
-// Scratch for lf_block_sparse_attn_noalloc: a fixed-size array in device global memory
-// that every device loading this library holds until the process exits.  Host code
-// must not use the symbol itself as a device address; the device address is obtained
-// once per device with cudaGetSymbolAddress (with that device current) and cached.
+// Scratch for lf_block_sparse_attn_noalloc: a fixed-size array in device global memory.
+// It exists on a device once this library's module is loaded there (with lazy module
+// loading, at the first use of the library on that device) and lives until the context
+// is destroyed.  Host code must not use the symbol itself as a device address: the address
+// is looked up with cudaGetSymbolAddress, with the device current, and cached together
+// with the context it belongs to, so that a context re-created after cudaDeviceReset (the
+// module reloaded, possibly at another address) gets a fresh lookup.
 constexpr size_t kNoAllocScratchBytes = 16u << 20;       // 16 MiB
 static __device__ __align__(256) uint8_t g_lf_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
+struct ScratchAddr {
+  CUcontext ctx;
+  void* addr;
+};
+ScratchAddr g_noalloc_addr[kMaxDevices] = {};
 
-// Device address of the fixed scratch on the current device (set up on first use).
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+std::once_flag g_ctx_once;
+
+// The current context of the calling thread (the runtime's primary context once any
+// runtime call has initialised the device), or null if it cannot be read.
+CUcontext current_context() {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  });
+  CUcontext c = nullptr;
+  if (g_ctx_current == nullptr || g_ctx_current(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of the fixed scratch on the current device and context (looked up on
+// the first call in that context).
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  ScratchAddr& e = g_noalloc_addr[dev];
+  const CUcontext ctx = current_context();       // null before the runtime's first use
+  if (ctx == nullptr || e.addr == nullptr || e.ctx != ctx) {
     void* p = nullptr;
+    // the lookup itself makes the device's primary context current
     if (cudaGetSymbolAddress(&p, g_lf_noalloc_scratch) != cudaSuccess || p == nullptr)
       return LF_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
+    const CUcontext now = current_context();
+    if (now == nullptr) return LF_ERR_CUDA;
+    e.ctx = now;
+    e.addr = p;
   }
-  *out = g_noalloc_addr[dev];
+  *out = e.addr;
   return LF_OK;
 }
 
@@ -692,11 +729,12 @@ int lf_select_chunk_cached(const lf_shape* shape, const void* q, const float* k_
                             stream);
 }
 
-int lf_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {
-  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return LF_ERR_INVALID_ARG;
-  if (n == 0) return LF_OK;
-  lf::exp2_poly_kernel<<<lf::cdiv(n, 256), 256, 0, stream>>>(x, y, n);
-  return cuda_status(cudaGetLastError());
+int lf_debug_configure(uint64_t wait_limit_ns, int stall, int tail_split) {
+  if (wait_limit_ns > 10ull * lf::kWaitLimitNs) return LF_ERR_INVALID_ARG;
+  g_dbg_wait_limit_ns = wait_limit_ns == 0 ? lf::kWaitLimitNs : wait_limit_ns;
+  g_dbg_stall = stall != 0;
+  g_dbg_tail_split = tail_split != 0;
+  return LF_OK;
 }
 
 #ifdef LF_TRACE

@@ -262,6 +262,9 @@ struct AttnParams {
   int pieces;
   float* part_o;       // [n_tail * pieces, 128, d] unnormalised O
   float* part_ml;      // [n_tail * pieces, 2, 128] row max (log2 units) and row sum
+  uint64_t wait_limit_ns;     // limit of every bounded wait of the launch (kWaitLimitNs)
+  int debug_stall;     // test hook: when set, CTA 0 never arms its Q barrier, so its
+                       // first wait runs out (the timeout and drain path)
   int slots[LF_MAX_FRAMES];   // cache slot of frame position p (sinks, then history)
 };
 
@@ -308,52 +311,6 @@ constexpr int kSoftmaxWarps = 8;          // two warpgroups, alternate key tiles
 // registers to the two softmax warpgroups: 128 x 72 + 256 x 216 <= 384 x 168.
 constexpr int kLaunchRegs = 168, kLowRegs = 72, kHighRegs = 216;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kAttnThreads * kLaunchRegs, "register split");
-
-// 2^x on the FMA pipe for x <= 8 (a share of the softmax exponentials is computed here
-// to unload the special-function unit).  Range reduction x = j + f, j = round(x),
-// f in [-1/2, 1/2], by adding and subtracting 1.5 * 2^23; 2^f by a degree-3 polynomial
-// (minimax relative error 7.5e-5, Remez fit, see gen_exp2_poly.py); j is added to the
-// IEEE-754 exponent field.  x is clamped at -126 so that the exponent field cannot go
-// below zero: -inf (a masked logit) gives about 1.2e-38.  Two lanes per instruction.
-constexpr float kExpC0 = 0.999928057f, kExpC1 = 0.693260968f, kExpC2 = 0.242611125f,
-                kExpC3 = 0.0551716685f, kShifter = 12582912.0f;
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 t = fadd2(x, make_float2(kShifter, kShifter));
-  const float2 j = fadd2(t, make_float2(-kShifter, -kShifter));
-  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);
-  float2 p = ffma2(make_float2(kExpC3, kExpC3), f, make_float2(kExpC2, kExpC2));
-  p = ffma2(p, f, make_float2(kExpC1, kExpC1));
-  p = ffma2(p, f, make_float2(kExpC0, kExpC0));
-  // bits(p) + (bits(t) << 23): the low bits of t hold j (two's complement)
-  return make_float2(__int_as_float(__float_as_int(p.x) + (int)((uint32_t)__float_as_int(t.x) * 8388608u)),
-                     __int_as_float(__float_as_int(p.y) + (int)((uint32_t)__float_as_int(t.y) * 8388608u)));
-}
-
-__device__ __forceinline__ float exp2_poly(float x) {
-  return exp2_poly2(make_float2(x, x)).x;
-}
-
-__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = exp2_poly(x[i]);
-}
-
-// How many of every 8 consecutive key pairs take the polynomial (tuning knob; 0 measured
-// fastest on B200 for this kernel, where the softmax is bound by its per-tile latency
-// chain rather than by the special-function unit).
-#ifndef LF_EXP2_FMA_PAIRS_OF_8
-#define LF_EXP2_FMA_PAIRS_OF_8 0
-#endif
-__host__ __device__ constexpr bool pair_on_fma(int e) {
-  return LF_EXP2_FMA_PAIRS_OF_8 == 0 ? false
-       : LF_EXP2_FMA_PAIRS_OF_8 == 1 ? (e & 7) == 5
-       : LF_EXP2_FMA_PAIRS_OF_8 == 2 ? ((e & 7) == 2 || (e & 7) == 6)
-       : LF_EXP2_FMA_PAIRS_OF_8 == 3 ? ((e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7)
-       : (e & 1) == 1;
-}
 
 template <int HD, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -436,12 +393,14 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   if (warp == 0 && lane == 0) {
     uint64_t* full = &bars[kBarRing];
     uint64_t* empty = &bars[kBarRing + L::kSlots];
-    mbar_arrive_expect_tx(&bars[kBarQ], L::kQBytes);
-    for (int c = 0; c < L::NH; ++c) {
-      uint8_t* dst = smem + L::kQ + c * L::kRegion;
-      tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD + c * 64, tokA);
-      tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD + c * 64,
-                  BLK == 64 ? tokB : tokA + 64);
+    if (!(P.debug_stall && blockIdx.x == 0)) {
+      mbar_arrive_expect_tx(&bars[kBarQ], L::kQBytes);
+      for (int c = 0; c < L::NH; ++c) {
+        uint8_t* dst = smem + L::kQ + c * L::kRegion;
+        tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD + c * 64, tokA);
+        tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD + c * 64,
+                    BLK == 64 ? tokB : tokA + 64);
+      }
     }
     const int n_pos = 2 * n_iter + 1;               // V of the last tile sits at 2n
     int q = 0;
@@ -451,7 +410,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       const int slot = q % L::kSlots;
       const int rnd = q / L::kSlots;
       if (isK && l >= n_iter) continue;            // no slot used, nothing to load
-      if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort)) break;
+      if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort, P.wait_limit_ns)) break;
       const int j = j0 + l;
       LF_TR(isK ? 0 : 1, l);
       mbar_arrive_expect_tx(&full[slot], L::kStageBytes);
@@ -484,7 +443,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     for (int x = max(0, q - L::kSlots); x < q; ++x) {
       bool isK;
       const int lx = ring_tile(x, isK);
-      if (!(isK && lx >= n_iter)) mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1);
+      if (!(isK && lx >= n_iter)) mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1, P.wait_limit_ns);
     }
   }
   // -------------------------------------------------------------- MMA issuer
@@ -502,7 +461,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       const int s = l & 1;
       const int q = ring_pos_k(l), slot = q % L::kSlots;
       LF_TR(2, l);
-      if (!mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort)) return false;
+      if (!mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort, P.wait_limit_ns)) return false;
       LF_TR(3, l);
       tc_fence_after();
       const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
@@ -517,20 +476,20 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       mma_commit(&empty[slot]);
       return true;
     };
-    bool ok = mbar_wait(&bars[kBarQ], 0, s_abort);
+    bool ok = mbar_wait(&bars[kBarQ], 0, s_abort, P.wait_limit_ns);
     if (ok) ok = issue_s(0);
     if (ok && n_iter > 1) ok = issue_s(1);
     for (int l = 0; ok && l < n_iter; ++l) {
       const int s = l & 1;
       const int qv = ring_pos_v(l), vslot = qv % L::kSlots;
-      ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort);
+      ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort, P.wait_limit_ns);
       LF_TR(4, l);
       const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
       const uint32_t o_tmem = tmem + (s ? L::kColO1 : L::kColO0);
       // P arrives in two halves (keys 0-63, 64-127); each half's four MMAs go as soon
       // as it is written
       for (int hf = 0; ok && hf < 2; ++hf) {
-        ok = mbar_wait(&bars[kBarPFull + 2 * s + hf], (l >> 1) & 1, s_abort);
+        ok = mbar_wait(&bars[kBarPFull + 2 * s + hf], (l >> 1) & 1, s_abort, P.wait_limit_ns);
         if (!ok) break;
         if (hf == 0) LF_TR(5, l);
         tc_fence_after();
@@ -567,7 +526,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     for (int l = wg; l < n_iter; l += 2, ++n_mine) {
       const int j = j0 + l;
       if (threadIdx.x == 128) LF_TR(6, l);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + wg], (l >> 1) & 1, s_abort)) && ok;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + wg], (l >> 1) & 1, s_abort, P.wait_limit_ns)) && ok;
       if (threadIdx.x == 128) LF_TR(7, l);
       tc_fence_after();
       float sv[128];
@@ -660,12 +619,8 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
               const int i0 = ch * 32 + 2 * e;
               const float2 x = ffma2(make_float2(sv[i0], sv[i0 + 1]), c2, nm2);
               float2 p;
-              if (pair_on_fma(ch * 16 + e)) {
-                p = exp2_poly2(x);
-              } else {
-                p.x = ex2_approx(x.x);
-                p.y = ex2_approx(x.y);
-              }
+              p.x = ex2_approx(x.x);
+              p.y = ex2_approx(x.y);
               if (e & 1) ps1 = fadd2(ps1, p); else ps0 = fadd2(ps0, p);
               __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
               pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&b2));
@@ -686,7 +641,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       m_run = m_new;
       if (threadIdx.x == 128) LF_TR(11, l);
     }
-    ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0, s_abort)) && ok;
+    ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarDone], 0, s_abort, P.wait_limit_ns)) && ok;
     // merge the two groups' partial softmax states: O = sum_w 2^(m_w - m) O_w / l
     s_red[wg * 128 + r] = m_run;
     s_red[256 + wg * 128 + r] = l_run;
@@ -760,7 +715,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   if (threadIdx.x == 0) LF_TR_CTA(2, globaltimer_ns());
   if (warp == 1) {
     // everything the MMA thread issued is complete before tensor memory is released
-    if (lane == 0) mbar_wait_drain(&bars[kBarDone], 0);
+    if (lane == 0) mbar_wait_drain(&bars[kBarDone], 0, P.wait_limit_ns);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);

@@ -124,9 +124,10 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Bounded wait: returns false (and records LF_ERR_TIMEOUT) if the phase with the given
 // parity has not completed within `limit_ns`.  `*abort` short-cuts every later wait of
 // the CTA once one of them has timed out.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s, the default limit of a launch
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   if (*abort) return false;
   uint64_t t0 = globaltimer_ns();
@@ -134,7 +135,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 255u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         record_status(LF_ERR_TIMEOUT);
         return false;
@@ -145,11 +146,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Bounded wait that ignores the CTA abort flag: used to drain asynchronous copies and
 // MMAs before a CTA releases its shared and tensor memory.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       record_status(LF_ERR_TIMEOUT);
       return false;
     }

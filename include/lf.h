@@ -195,12 +195,14 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
  * no device allocation after start-up (cudaMalloc may synchronise the device).  This
  * entry point takes the same arguments minus the workspace and uses instead a fixed
  * scratch array in device global memory that lives in the library: at most
- * lf_noalloc_scratch_bytes() bytes (16 MiB), reserved on every device that loads the
- * library until the process exits.  It allocates nothing and calls no allocating routine.
+ * lf_noalloc_scratch_bytes() bytes (16 MiB), reserved on a device once the library's
+ * module is loaded there (with lazy module loading, at its first use on that device) and
+ * held until the process exits.  It allocates nothing and calls no allocating routine.
  *
  *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *    with that device current) and caches it; make that first call before any stream
- *    capture on the device.
+ *    with that device current) and caches it with the current context; a call in a new
+ *    context (after cudaDeviceReset) looks it up again.  Make the first call on a device
+ *    before any stream capture on it.
  *  - All calls on a device share the one array, which keeps the last call's contents
  *    (nothing in it needs to start at zero).  Calls whose work may overlap on the GPU —
  *    on different streams, or from different host threads — race on it; serialise them.
@@ -226,11 +228,20 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
                      void* workspace, size_t workspace_bytes, void* out, float* lse,
                      int32_t* block_idx_out, cudaStream_t stream);
 
-/* Test hook, not part of the attention path: evaluates the FMA-pipe exponential the
- * attention softmax uses for part of its probabilities, y[i] = 2^x[i] for x[i] <= 8
- * (degree-3 polynomial after round-to-nearest range reduction; relative error below
- * 1e-4 for -125 <= x <= 8; x below -126 gives about 1.2e-38).  x, y: device fp32 [n]. */
-int lf_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+/* Test hook, not part of the attention path (process-wide, not thread-safe; call it only
+ * while no library work is queued).  Sets, for the attention launches that follow:
+ *   wait_limit_ns  the limit of every bounded device wait (0 = the default, 2 s; at most
+ *                  20 s);
+ *   stall          nonzero: the first CTA of each attention launch never arms its query
+ *                  barrier, so its waits run out after wait_limit_ns; the launch then
+ *                  drains, frees its tensor memory, returns, and lf_device_status()
+ *                  reports LF_ERR_TIMEOUT (that launch's output is undefined);
+ *   tail_split     zero: every query tile is computed whole (no split of the last partial
+ *                  wave into key ranges), so each tile's rounding is independent of how
+ *                  many tiles a launch has.
+ * lf_debug_configure(0, 0, 1) restores the defaults.  LF_ERR_INVALID_ARG for a limit
+ * above 20 s. */
+int lf_debug_configure(uint64_t wait_limit_ns, int stall, int tail_split);
 
 /* Chunk-aware growth of the sparsity [LF-gist 2.1, consistency-aware growth]: the sparsity
  * of chunk i rises as the noise level alpha_i falls, s_i = s_base - alpha_i * beta, here

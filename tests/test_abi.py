@@ -141,3 +141,9 @@ def test_select_1d_block_limit(lib):
     h4, _k2 = _i32([0, 1, 2, 3])
     assert lib.lf_select_chunk_1d(ctypes.byref(small), FAKE, FAKE, h4, FAKE, None, 0,
                                   None) == 5
+
+
+def test_debug_configure_validates_and_restores(lib):
+    assert lib.lf_debug_configure(30_000_000_000, 0, 1) == 1          # above 20 s
+    assert lib.lf_debug_configure(20_000_000, 0, 0) == 0
+    assert lib.lf_debug_configure(0, 0, 1) == 0                       # defaults

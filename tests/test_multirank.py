@@ -74,18 +74,27 @@ def test_shard_heads_is_a_head_slice():
 
 
 def test_oracle_timings_are_bounded_samples():
-    """The CPU-baseline helpers: one head per sample without a budget, the torch thread
-    count restored after the single-thread run, the FLOPs those of the heads run."""
+    """The CPU-baseline helpers: one (chunk, head) unit per sample without a budget, the
+    torch thread count restored after the single-thread run, the FLOPs those of the units
+    run; a workload of several chunks is sampled across its chunks in order."""
     import lf_workloads as W
     ci = W.tiny(0)
     n = torch.get_num_threads()
-    f, dt, cores, heads = bench.oracle_sample(ci)
-    assert heads == 1 and f > 0 and dt > 0 and cores == n
-    f1, dt1 = bench.oracle_single_core(ci)
+    f, dt, cores, units = bench.oracle_sample([ci])
+    assert units == 1 and f > 0 and dt > 0 and cores == n
+    f1, dt1 = bench.oracle_single_core([ci])
     assert f1 == f and dt1 > 0
     assert torch.get_num_threads() == n
-    f_all, _, _, heads_all = bench.oracle_sample(ci, budget_s=1e9)
-    assert heads_all == ci.shape.H and f_all == ci.shape.H * f
+    f_all, _, _, units_all = bench.oracle_sample([ci], budget_s=1e9)
+    assert units_all == ci.shape.H and f_all == ci.shape.H * f
+    ci2 = W.tiny(1)
+    f2, _, _, u2 = bench.oracle_sample([ci, ci2], budget_s=1e9)
+    g2, _, _, _ = bench.oracle_sample([ci2], budget_s=1e9)
+    assert u2 == 2 * ci.shape.H and f2 == f_all + g2
+    # starting at unit H runs the second chunk's first head
+    f_b, _, _, _ = bench.oracle_sample([ci, ci2], first=ci.shape.H)
+    f_c, _, _, _ = bench.oracle_sample([ci2])
+    assert f_b == f_c
 
 
 def test_clock_summary_from_fake_rows():

@@ -34,6 +34,9 @@ def _inputs(ci):
                                                          n_cur_frames=2, n_hist=3, n_sink=1,
                                                          k_f=2, k_b=2)])
 def test_noalloc_matches_workspace_entry_point_twice(gpu_lib, make):
+    """Same kernels, same inputs: the outputs and lse must be the same bits as those of
+    lf_block_sparse_attn with a caller workspace, on two calls in a row (the second call
+    finds the first call's contents in the shared scratch)."""
     ci = make()
     sh = ci.shape
     t, bidx = _inputs(ci)
@@ -49,8 +52,14 @@ def test_noalloc_matches_workspace_entry_point_twice(gpu_lib, make):
                                              t["v_cache"], ci.hist_slots, ci.sink_slots, bidx,
                                              out, lse)
         torch.cuda.synchronize()
-        G.assert_output_close(out, ref.float().cpu().double().numpy(), what="noalloc")
-        assert torch.allclose(lse, ref_lse, rtol=0, atol=G.LSE_ABS)
+        assert torch.equal(out, ref), "output differs from lf_block_sparse_attn"
+        assert torch.equal(lse, ref_lse), "lse differs from lf_block_sparse_attn"
+    if ci.shape.H * ci.shape.T <= 1024:      # the tiny shape: also against the float64 oracle
+        o_ref, lse_ref = O.attention(sh, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                                     ci.hist_slots, ci.sink_slots,
+                                     None if bidx is None else bidx.cpu().numpy())
+        G.assert_output_close(out, o_ref, what="noalloc vs oracle")
+        assert np.abs(lse.cpu().double().numpy() - lse_ref).max() <= G.LSE_ABS
     assert gpu_lib.lf_device_status() == 0
 
 
