@@ -44,6 +44,7 @@ class Shape:
     k_f: int               # frames kept per query block
     k_b: int               # blocks kept per chosen frame
     scale: float           # softmax scale (1/sqrt(d))
+    k_c: int = 0           # current-chunk blocks kept per query block (0: dense)
 
 
 @dataclass
@@ -182,13 +183,13 @@ def large(seed: int = 0, n_hist: Optional[int] = None) -> ChunkInputs:
 
 def random_small(seed: int, H: int, d: int, T: int, block: int, n_cur_frames: int,
                  n_hist: int, n_sink: int, k_f: int, k_b: int,
-                 extra_slots: int = 1) -> ChunkInputs:
+                 extra_slots: int = 1, k_c: int = 0) -> ChunkInputs:
     """Small random shape for parity sweeps: centroids N(0, 0.5), planted queries, and a
     cache with spare slots (unused slots are filled too, so a wrong slot id shows)."""
     n_slots = n_hist + n_sink + extra_slots
     shape = Shape(H=H, d=d, T=T, block=block, n_cur_frames=n_cur_frames, n_hist=n_hist,
                   n_sink=n_sink, n_slots=n_slots, k_f=k_f, k_b=k_b,
-                  scale=1.0 / float(np.sqrt(d)))
+                  scale=1.0 / float(np.sqrt(d)), k_c=k_c)
     ci = _centroid_chunk(shape, seed, f"rand{seed}", 0.5, 0.5, True,
                          slot_start=seed % max(n_slots - n_sink, 1))
     g = _streams(seed + 1000, 1)[0]

@@ -31,6 +31,9 @@ unscaled dot products; top-k keeps the k largest, ties going to the lower index,
 index lists are returned ascending; k_b blocks are kept in EACH chosen frame; the current
 chunk and the sink frames are always attended densely and are never candidates; the
 softmax is one joint softmax over current + sink + selected keys with scale 1/sqrt(d).
+Optionally (k_c > 0) the current chunk is sparse too: its keys are mean-pooled per block
+like the queries, and each query block keeps its own block plus the k_c - 1 other
+current-chunk blocks with the largest q_blk . k_blk (ties to the lower index).
 
 All arithmetic is float64 on values upcast from the bf16 inputs.
 """
@@ -45,7 +48,7 @@ __all__ = [
     "block_bounds", "n_blocks", "compress_queries", "compress_keys", "frame_scores",
     "topk_lower_index", "select_frames", "block_scores_in_frame", "select_blocks",
     "key_set", "attention_qblock", "attention", "forward_chunk", "boundary_gap",
-    "select_blocks_1d", "executed_flops",
+    "select_blocks_1d", "select_current_blocks", "current_boundary_gap", "executed_flops",
 ]
 
 
@@ -191,15 +194,51 @@ def select_blocks_1d(q_blk: np.ndarray, k_blk: np.ndarray, k: int):
     return idx, s
 
 
+def select_current_blocks(q_blk: np.ndarray, kc_blk: np.ndarray, k_c: int):
+    """[LF-yly 一, second scenario: 80% sparsity applied to the first chunk, which has no
+    history, so the sparsity reaches the current chunk's own keys; LF-gist 2.2, token
+    compression and block selection by inner products.]  Reading: the current chunk's keys
+    are mean-pooled per block exactly as its queries are (kc_blk = compress_queries(k_cur));
+    query block qb keeps its own block qb (the diagonal) and the k_c - 1 other current
+    blocks with the largest scores q_blk[h, qb] . kc_blk[h, c], equal scores to the lower
+    index.  Returns cur_idx [H, n_qb, min(k_c, n_qb)] ascending and the scores
+    [H, n_qb, n_qb] of every current block."""
+    H, nqb, _ = q_blk.shape
+    kk = min(k_c, nqb)
+    idx = np.empty((H, nqb, kk), dtype=np.int64)
+    sc = np.empty((H, nqb, nqb))
+    for h in range(H):
+        for qb in range(nqb):
+            sc[h, qb] = block_scores_in_frame(q_blk[h, qb], kc_blk[h])
+            others = [c for c in range(nqb) if c != qb]
+            best = topk_lower_index([sc[h, qb, c] for c in others], kk - 1)
+            idx[h, qb] = sorted([qb] + [others[i] for i in best])
+    return idx, sc
+
+
+def current_boundary_gap(scores: Sequence[float], own: int, k_c: int) -> float:
+    """boundary_gap of the current-chunk choice of one query block: the own block is
+    always kept, so the gap is that of the k_c - 1 best among the other blocks."""
+    return boundary_gap([x for c, x in enumerate(scores) if c != own], k_c - 1)
+
+
 def key_set(shape, qb_blocks: Sequence[int], cur_h: np.ndarray, cache_h: np.ndarray,
-            hist_slots, sink_slots) -> np.ndarray:
-    """Keys (or values) one query block attends to, in a fixed order: the whole current
-    chunk (dense), every token of every sink frame, then the tokens of the selected
-    history blocks.  cur_h: [F_c*T, d] and cache_h: [n_slots, T, d] are one head's
-    float64 tensors.  Returns [n_keys, d]."""
+            hist_slots, sink_slots, cur_blocks=None) -> np.ndarray:
+    """Keys (or values) one query block attends to, in a fixed order: the current chunk
+    (every token, or with `cur_blocks` the tokens of those current-chunk blocks, block
+    qb = frame * n_bpf + b), every token of every sink frame, then the tokens of the
+    selected history blocks.  cur_h: [F_c*T, d] and cache_h: [n_slots, T, d] are one
+    head's float64 tensors.  Returns [n_keys, d]."""
     bounds = block_bounds(shape.T, shape.block)
     nb = len(bounds)
-    parts = [cur_h]
+    if cur_blocks is None:
+        parts = [cur_h]
+    else:
+        parts = []
+        for c in cur_blocks:
+            f, b = divmod(int(c), nb)
+            s, e = bounds[b]
+            parts.append(cur_h[f * shape.T + s: f * shape.T + e])
     for slot in sink_slots:
         parts.append(cache_h[slot])
     for g in qb_blocks:
@@ -221,11 +260,13 @@ def attention_qblock(q_rows: np.ndarray, keys: np.ndarray, values: np.ndarray, s
 
 
 def attention(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
-              block_idx, heads=None, qblocks=None):
+              block_idx, heads=None, qblocks=None, cur_idx=None):
     """[LF-gist 2.2 / LF-yly 三, block-sparse attention; SF rolling cache; RF sinks]
     For each query token of query block qb, one joint softmax over the current chunk's
-    keys, the sink frames' keys and the keys of qb's selected history blocks.
+    keys (all of them, or with cur_idx only those of qb's kept current blocks), the sink
+    frames' keys and the keys of qb's selected history blocks.
     block_idx: [H, n_qb, n_sel] global block ids (ignored when there is no history).
+    cur_idx: None (dense current chunk) or [H, n_qb, n_c] current-chunk block ids.
     Returns O [F_c*T, H, d] and lse [H, F_c*T] (natural log of the scaled-logit
     normaliser); entries outside ``heads`` x ``qblocks`` are left as NaN."""
     T, B = shape.T, shape.block
@@ -246,8 +287,9 @@ def attention(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
             s, e = bounds[b]
             rows = slice(f * T + s, f * T + e)
             sel = [] if len(hist_slots) == 0 else list(block_idx[h, qb])
-            keys = key_set(shape, sel, kcur_h, kc_h, hist_slots, sink_slots)
-            vals = key_set(shape, sel, vcur_h, vc_h, hist_slots, sink_slots)
+            cur = None if cur_idx is None else list(cur_idx[h, qb])
+            keys = key_set(shape, sel, kcur_h, kc_h, hist_slots, sink_slots, cur)
+            vals = key_set(shape, sel, vcur_h, vc_h, hist_slots, sink_slots, cur)
             o, l, _ = attention_qblock(qf[rows, h, :], keys, vals, shape.scale)
             O[rows, h, :] = o
             lse[h, rows] = l
@@ -255,31 +297,42 @@ def attention(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
 
 
 def forward_chunk(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots):
-    """(a) compress -> (b) frame top-k -> (c) block top-k -> (d) block-sparse attention."""
+    """(a) compress -> (b) frame top-k -> (c) block top-k -> (d) block-sparse attention.
+    With shape.k_c > 0 (default 0: dense current chunk) the current chunk's blocks are
+    selected too (select_current_blocks) and attended sparsely."""
     out = {}
-    if len(hist_slots) > 0:
+    k_c = getattr(shape, "k_c", 0)
+    if len(hist_slots) > 0 or k_c > 0:
         q_blk = compress_queries(q, shape.T, shape.block)
+        out.update(q_blk=q_blk)
+    if len(hist_slots) > 0:
         k_blk, k_frm = compress_keys(k_cache, hist_slots, shape.T, shape.block)
         frame_idx, sf = select_frames(q_blk, k_frm, shape.k_f)
         block_idx, sb = select_blocks(q_blk, k_blk, frame_idx, shape.k_b)
-        out.update(q_blk=q_blk, k_blk=k_blk, k_frm=k_frm, frame_idx=frame_idx,
+        out.update(k_blk=k_blk, k_frm=k_frm, frame_idx=frame_idx,
                    frame_scores=sf, block_idx=block_idx, block_scores=sb)
     else:
         block_idx = None
+    cur_idx = None
+    if k_c > 0:
+        kc_blk = compress_queries(k_cur, shape.T, shape.block)
+        cur_idx, sc = select_current_blocks(q_blk, kc_blk, k_c)
+        out.update(kc_blk=kc_blk, cur_idx=cur_idx, cur_scores=sc)
     O, lse = attention(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
-                       block_idx)
+                       block_idx, cur_idx=cur_idx)
     out.update(O=O, lse=lse)
     return out
 
 
 # ------------------------------------------------------------ algorithmic work
-def executed_flops(shape, block_idx) -> int:
-    """4*d per (head, query, valid key) pair: the QK^T and PV products actually needed."""
+def executed_flops(shape, block_idx, cur_idx=None) -> int:
+    """4*d per (head, query, valid key) pair: the QK^T and PV products actually needed
+    (the current chunk dense, or only the kept current blocks when cur_idx is given)."""
     T, B = shape.T, shape.block
     bounds = block_bounds(T, B)
     nb = len(bounds)
     Fc = shape.n_cur_frames
-    dense_keys = Fc * T + shape.n_sink * T
+    dense_keys = (Fc * T if cur_idx is None else 0) + shape.n_sink * T
     total = 0
     for h in range(shape.H):
         for qb in range(Fc * nb):
@@ -289,6 +342,9 @@ def executed_flops(shape, block_idx) -> int:
                 for g in block_idx[h, qb]:
                     bs, be = bounds[int(g) % nb]
                     nsel += be - bs
+            if cur_idx is not None:
+                for c in cur_idx[h, qb]:
+                    bs, be = bounds[int(c) % nb]
+                    nsel += be - bs
             total += (e - s) * (dense_keys + nsel)
     return 4 * shape.d * total
-

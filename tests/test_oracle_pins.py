@@ -396,6 +396,157 @@ def test_select_blocks_1d_degenerate_and_two_stage():
     assert np.array_equal(one_d, two)
 
 
+# ------------------------------------------------------------------ sparse current chunk
+@pytest.mark.parametrize("seed", range(12))
+def test_current_selection_brute_force(seed):
+    """Own block always kept, plus the (k_c - 1)-subset of the other current blocks with the
+    largest score sum (scores recomputed here as plain dot products), lexicographically
+    smallest among equal sums; the own block is kept even when it scores lowest."""
+    g = np.random.default_rng(200 + seed)
+    H, nqb, d = 2, int(g.integers(1, 8)), 6
+    q = g.standard_normal((H, nqb, d))
+    kc = g.standard_normal((H, nqb, d))
+    if seed % 3 == 1 and nqb > 2:           # exact ties between other blocks
+        kc[:, 2] = kc[:, 1]
+    if seed % 3 == 2:                       # small integers: many exact ties everywhere
+        q = g.integers(-1, 2, size=(H, nqb, d)).astype(float)
+        kc = g.integers(-1, 2, size=(H, nqb, d)).astype(float)
+    k = int(g.integers(1, nqb + 2))          # also k_c > n_qb
+    idx, sc = O.select_current_blocks(q, kc, k)
+    kk = min(k, nqb)
+    assert idx.shape == (H, nqb, kk)
+    for h in range(H):
+        for qq in range(nqb):
+            flat = [float(np.dot(q[h, qq], kc[h, c])) for c in range(nqb)]
+            assert np.allclose(sc[h, qq], flat, rtol=0, atol=1e-12)
+            others = [c for c in range(nqb) if c != qq]
+            best = _brute_topk([flat[c] for c in others], kk - 1) if kk > 1 else []
+            assert list(idx[h, qq]) == sorted([qq] + [others[i] for i in best])
+
+
+def test_current_selection_keeps_own_block_when_it_scores_lowest():
+    q = np.ones((1, 3, 2))
+    kc = np.array([[[-5.0, -5.0], [1.0, 0.0], [2.0, 0.0]]])     # block 0 scores -10
+    idx, _ = O.select_current_blocks(q, kc, 2)
+    assert idx[0].tolist() == [[0, 2], [1, 2], [1, 2]]
+    assert O.current_boundary_gap([-10.0, 1.0, 2.0], 0, 2) == pytest.approx(0.5)
+
+
+@pytest.mark.parametrize("T,B,F,S", [(100, 32, 3, 0), (64, 64, 2, 1)])
+def test_current_all_kept_equals_dense(T, B, F, S):
+    """k_c >= n_qb keeps every current block: the same result as the dense current chunk
+    (the same keys in the same order) and as plain SDPA when all history is kept too."""
+    nbpf = -(-T // B)
+    ci = W.random_small(T + 5, H=2, d=16, T=T, block=B, n_cur_frames=2, n_hist=F,
+                        n_sink=S, k_f=F, k_b=nbpf)
+    dense = O.forward_chunk(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                            ci.hist_slots, ci.sink_slots)
+    from dataclasses import replace
+    sparse = O.forward_chunk(replace(ci.shape, k_c=2 * nbpf + 3), ci.q, ci.k_cur, ci.v_cur,
+                             ci.k_cache, ci.v_cache, ci.hist_slots, ci.sink_slots)
+    assert np.array_equal(sparse["O"], dense["O"]) and np.array_equal(sparse["lse"], dense["lse"])
+    assert sparse["cur_idx"].tolist() == [[list(range(2 * nbpf))] * (2 * nbpf)] * 2
+    o_ref, lse_ref = _dense_reference_sdpa(ci)
+    assert np.allclose(sparse["O"], o_ref, rtol=0, atol=1e-12)
+
+
+def _masked_reference_sdpa_cur(ci, block_idx, cur_idx):
+    """SDPA with a token mask over the current chunk too: a current key token t is visible
+    to a query token iff block (t // T) * n_bpf + (t % T) // B is in the query block's
+    current list; sinks always; history tokens as in _masked_reference_sdpa."""
+    sh = ci.shape
+    T, B, Fc = sh.T, sh.block, sh.n_cur_frames
+    nbpf = -(-T // B)
+    keys = [ci.k_cur.double()] + [ci.k_cache[s].double() for s in ci.sink_slots] + \
+           [ci.k_cache[s].double() for s in ci.hist_slots]
+    vals = [ci.v_cur.double()] + [ci.v_cache[s].double() for s in ci.sink_slots] + \
+           [ci.v_cache[s].double() for s in ci.hist_slots]
+    K = torch.cat(keys, 0).permute(1, 0, 2)
+    V = torch.cat(vals, 0).permute(1, 0, 2)
+    Q = ci.q.double().permute(1, 0, 2)
+    n_q, n_dense = Fc * T, Fc * T + sh.n_sink * T
+    tq = torch.arange(n_q)
+    q_block = (tq // T) * nbpf + (tq % T) // B
+    th = torch.arange(sh.n_hist * T)
+    k_block = (th // T) * nbpf + (th % T) // B
+    mask = torch.ones(sh.H, n_q, n_dense + sh.n_hist * T, dtype=torch.bool)
+    for h in range(sh.H):
+        cur = torch.zeros(Fc * nbpf, Fc * nbpf, dtype=torch.bool)
+        for qb in range(Fc * nbpf):
+            cur[qb, torch.as_tensor(cur_idx[h, qb], dtype=torch.long)] = True
+        mask[h, :, :n_q] = cur[q_block][:, q_block]
+        if sh.n_hist > 0:
+            sel = torch.zeros(Fc * nbpf, sh.n_hist * nbpf, dtype=torch.bool)
+            for qb in range(Fc * nbpf):
+                sel[qb, torch.as_tensor(block_idx[h, qb], dtype=torch.long)] = True
+            mask[h, :, n_dense:] = sel[q_block][:, k_block]
+    out = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None],
+                                                           attn_mask=mask[None],
+                                                           scale=sh.scale)[0]
+    logits = torch.einsum("hqd,hkd->hqk", Q, K) * sh.scale
+    lse = torch.logsumexp(logits.masked_fill(~mask, float("-inf")), -1)
+    return out.permute(1, 0, 2).numpy(), lse.numpy()
+
+
+@pytest.mark.parametrize("seed,T,B,F,S,nsel,ncur", [(31, 100, 32, 3, 0, 5, 3),
+                                                    (32, 70, 16, 0, 1, 0, 4),
+                                                    (33, 40, 64, 4, 2, 3, 1)])
+def test_sparse_current_equals_masked_sdpa(seed, T, B, F, S, nsel, ncur):
+    """Any current-chunk lists (random, each holding its own block) together with any
+    history lists give the attention of a token mask built from the lists."""
+    nbpf = -(-T // B)
+    ci = W.random_small(seed, H=2, d=16, T=T, block=B, n_cur_frames=2, n_hist=F,
+                        n_sink=S, k_f=1, k_b=1)
+    g = np.random.default_rng(seed)
+    nqb = 2 * nbpf
+    cur = np.stack([np.stack([np.sort(np.concatenate(
+        [[qb], g.choice([c for c in range(nqb) if c != qb], size=min(ncur, nqb) - 1,
+                        replace=False)]).astype(np.int64)) for qb in range(nqb)])
+        for _ in range(2)])
+    bidx = None
+    if F > 0:
+        bidx = np.stack([np.stack([np.sort(g.choice(F * nbpf, size=nsel, replace=False))
+                                   for _ in range(nqb)]) for _ in range(2)])
+    o, lse = O.attention(ci.shape, ci.q, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                         ci.hist_slots, ci.sink_slots, bidx, cur_idx=cur)
+    o_ref, lse_ref = _masked_reference_sdpa_cur(ci, bidx, cur)
+    assert np.allclose(o, o_ref, rtol=0, atol=1e-12)
+    assert np.allclose(lse, lse_ref, rtol=0, atol=1e-12)
+
+
+def test_current_own_block_only_closed_form():
+    """k_c = 1, no history, q = 0: every key of the own block and of the sinks has the
+    same logit, so O is the plain mean of those values and lse = log(their count)."""
+    ci = W.random_small(41, H=2, d=16, T=50, block=16, n_cur_frames=2, n_hist=0,
+                        n_sink=1, k_f=1, k_b=1, k_c=1)
+    sh = ci.shape
+    zq = torch.zeros_like(ci.q)
+    r = O.forward_chunk(sh, zq, ci.k_cur, ci.v_cur, ci.k_cache, ci.v_cache,
+                        ci.hist_slots, ci.sink_slots)
+    lens = [16, 16, 16, 2]
+    vc64 = ci.v_cur.double().numpy()
+    vs = ci.v_cache.double().numpy()[ci.sink_slots[0]]
+    for h in range(2):
+        for qb in range(8):
+            f, b = divmod(qb, 4)
+            rows = slice(f * 50 + b * 16, f * 50 + b * 16 + lens[b])
+            assert r["cur_idx"][h, qb].tolist() == [qb]
+            total = vc64[rows, h].sum(0) + vs[:, h].sum(0)
+            n_keys = lens[b] + 50
+            assert np.allclose(r["O"][rows, h], total / n_keys, rtol=0, atol=1e-12)
+            assert np.allclose(r["lse"][h, rows], math.log(n_keys), rtol=0, atol=1e-12)
+
+
+def test_executed_flops_with_sparse_current():
+    """4*d per pair, with only the kept current blocks' tokens counted."""
+    ci = W.random_small(42, H=1, d=16, T=50, block=16, n_cur_frames=1, n_hist=0,
+                        n_sink=0, k_f=1, k_b=1)
+    cur = np.array([[[0, 3], [1, 3], [0, 2], [3, 2]]])      # lists need not be sorted here
+    lens = [16, 16, 16, 2]
+    expect = sum(lens[qb] * sum(lens[c] for c in cur[0, qb]) for qb in range(4))
+    assert O.executed_flops(ci.shape, None, cur) == 4 * 16 * expect
+
+
 # ------------------------------------------------------------------ chunk-aware growth
 @pytest.mark.parametrize("n,first,mean,final", [(7, 2, 0.8, 0.9), (20, 2, 0.8, 0.95),
                                                 (5, 3, 0.5, 0.6), (4, 1, 0.3, 0.2)])
