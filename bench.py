@@ -51,37 +51,57 @@ def block_lens(T, B):
     return np.array([min(B, T - b * B) for b in range(nb)], dtype=np.int64)
 
 
-def executed_flops(shape, block_idx_np) -> int:
-    """4*d per (head, query, valid key): current chunk + sinks dense, plus the tokens of the
-    selected blocks of each query's block."""
+def executed_flops(shape, block_idx_np, cur_idx_np=None) -> int:
+    """4*d per (head, query, valid key): current chunk (dense, or the kept current blocks
+    of each query's block) + sinks dense, plus the tokens of the selected history blocks."""
     lens = block_lens(shape.T, shape.block)
     nb = len(lens)
     qlen = np.tile(lens, shape.n_cur_frames)                  # tokens per query block
-    dense = shape.n_cur_frames * shape.T + shape.n_sink * shape.T
+    dense = (shape.n_cur_frames * shape.T if cur_idx_np is None else 0) + shape.n_sink * shape.T
     sel = np.zeros((shape.H, len(qlen)), dtype=np.int64)
     if shape.n_hist > 0 and block_idx_np is not None:
-        sel = lens[block_idx_np % nb].sum(axis=-1)
+        sel = sel + lens[block_idx_np % nb].sum(axis=-1)
+    if cur_idx_np is not None:
+        sel = sel + lens[cur_idx_np % nb].sum(axis=-1)
     return int(4 * shape.d * (qlen[None, :] * (dense + sel)).sum())
 
 
 def tail_split(shape, n_sm=148) -> bool:
     """Whether the attention launch splits its last, partial wave of tiles (mirrors the
-    library's rule: the last wave is less than half full)."""
-    tiles = shape.H * (-(-shape.n_cur_frames * -(-shape.T // shape.block) // (2 if shape.block == 64 else 1)))
+    library's rule: the last wave is less than half full, and it can be cut into at least
+    two key ranges of at least one key tile each)."""
+    per = 2 if shape.block == 64 else 1
+    nbpf = -(-shape.T // shape.block)
+    nqb = shape.n_cur_frames * nbpf
+    tiles = shape.H * -(-nqb // per)
     r = tiles % n_sm
-    return r != 0 and 2 * r <= n_sm
+    if r == 0 or 2 * r > n_sm:
+        return False
+    k_c = getattr(shape, "k_c", 0)
+    kc = min(k_c, nqb) if k_c > 0 else 0
+    nsel = (min(shape.k_f, shape.n_hist) * min(shape.k_b, nbpf)) if shape.n_hist > 0 else 0
+    min_tiles = (0 if kc > 0 else -(-shape.n_cur_frames * shape.T // 128)) + \
+        -(-(shape.n_sink * nbpf + kc + nsel) // per)
+    return min(n_sm // r, 16, min_tiles) >= 2
 
 
 def selection_launches(shape) -> int:
-    """Kernels one lf_select_chunk call launches (mirrors the library's rule): pooling,
-    block scores and pick when the fused path applies, else pooling, frame pooling, frame
-    selection and block selection."""
+    """Kernels one lf_select_chunk call launches (mirrors the library's rule): one when the
+    single-launch selection applies, else pooling, block scores and pick when the fused
+    path applies, else pooling, frame pooling, frame selection and block selection."""
     if shape.n_hist <= 0:
         return 0
     nbpf = -(-shape.T // shape.block)
+    nqb = shape.n_cur_frames * nbpf
     kf, kb = min(shape.k_f, shape.n_hist), min(shape.k_b, nbpf)
     fused = (shape.n_hist * nbpf <= 2048 and kf * kb <= 256 and shape.n_hist <= 256
              and nbpf <= 256)
+    pick_smem = 2 * shape.n_hist * nbpf * 4 + 2 * kf * kb * 4 + 2 * kf * 4
+    bb = 256 // (4 * (shape.d // 8))
+    stream_smem = max(bb * 4 * shape.d * 4 + 16 * (shape.d + 4) * 4 + nqb * (shape.d + 4) * 4,
+                      pick_smem)
+    if fused and getattr(shape, "k_c", 0) == 0 and stream_smem <= 227 * 1024:
+        return 1
     return 3 if fused else 4
 
 
@@ -225,7 +245,7 @@ def summarise_clocks(rows):
             "reasons": sorted(reasons), "samples": len(sm)}
 
 
-CONFIG_NAMES = ("480p", "large", "rolling", "growth")
+CONFIG_NAMES = ("480p", "large", "rolling", "growth", "chunk1_80")
 
 
 def make_workload(name, seed):
@@ -260,6 +280,15 @@ def make_workload(name, seed):
                        "(H=12 d=128 T=1560, B=64), history 0,3,...,18 frames, keep ratio " \
                        "1 then mean 0.2 over chunks 2-7 (k_f, k_b from lf_cag_schedule: " + \
                        ", ".join(f"({a},{b})" for a, b in zip(kf, kb)) + ")"
+    if name == "chunk1_80":
+        from dataclasses import replace
+        ci = W.growth_sweep(seed)[0]
+        nqb = ci.shape.n_cur_frames * -(-ci.shape.T // ci.shape.block)
+        k_c = nqb // 5                                       # keep 20%: 15 of 75 blocks
+        return [replace(ci, shape=replace(ci.shape, k_c=k_c), name="chunk1_80")], \
+            "first chunk at 80% sparsity inside the current chunk (no history): H=12 d=128 " \
+            f"T=1560, chunk 3 frames, B=64, each query block keeps its own block + the " \
+            f"{k_c - 1} best of the other {nqb - 1} current blocks"
     raise SystemExit(f"unknown config {name} (one of {', '.join(CONFIG_NAMES)})")
 
 
@@ -347,6 +376,8 @@ class ChunkRun:
         nbpf, nqb, kf, kb = lf.derived(sh)
         self.t = {k: getattr(ci, k).to(dev) for k in ("q", "k_cur", "v_cur", "k_cache", "v_cache")}
         self.bidx = torch.empty(sh.H, nqb, max(kf * kb, 1), dtype=torch.int32, device=dev)
+        self.kc = lf.current_blocks(sh)
+        self.cidx = torch.empty(sh.H, nqb, max(self.kc, 1), dtype=torch.int32, device=dev)
         self.sws = torch.empty(max(lf.lf_select_workspace_size(sh), 256), dtype=torch.uint8,
                                device=dev)
         self.out = torch.empty_like(self.t["q"])
@@ -355,20 +386,29 @@ class ChunkRun:
                               device=dev)
 
     def select(self):
+        t = self.t
         if self.sh.n_hist > 0:
-            t = self.t
             self.lf.lf_select_chunk(self.sh, t["q"], t["k_cache"], self.ci.hist_slots, self.bidx,
                                     self.sws)
+        if self.kc > 0:
+            self.lf.lf_select_current(self.sh, t["q"], t["k_cur"], self.cidx, self.sws)
 
     def attend(self):
         t = self.t
         self.lf.lf_block_sparse_attn(self.sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"],
                                      t["v_cache"], self.ci.hist_slots, self.ci.sink_slots,
-                                     self.bidx, self.out, self.lse, self.ws)
+                                     self.bidx, self.out, self.lse, self.ws,
+                                     cur_idx=self.cidx if self.kc > 0 else None)
+
+    def flops(self) -> int:
+        return executed_flops(self.sh, self.bidx.cpu().numpy(),
+                              self.cidx.cpu().numpy() if self.kc > 0 else None)
 
     def launches(self) -> int:
-        # selection kernels | plan, schedule, attn (+ merge)
-        return selection_launches(self.sh) + 3 + (1 if tail_split(self.sh) else 0)
+        # selection kernels (+ current-chunk pooling and choice) | plan, schedule, attn
+        # (+ merge)
+        return selection_launches(self.sh) + (2 if self.kc > 0 else 0) + 3 + \
+            (1 if tail_split(self.sh) else 0)
 
 
 def capture(fn, stream, cap):
@@ -447,7 +487,7 @@ def run_lf(args, rank, world, local_rank):
         flush_l2()
         step()
     torch.cuda.synchronize()
-    flops = sum(executed_flops(r.sh, r.bidx.cpu().numpy()) for r in runs)
+    flops = sum(r.flops() for r in runs)
     sel_bytes = sum(selection_bytes(r.sh) for r in runs if r.sh.n_hist > 0)
     launches_per_step = sum(r.launches() for r in runs)
 
@@ -481,7 +521,7 @@ def run_lf(args, rank, world, local_rank):
         job_flops = float(world * flops)
         value = weak_scaling_value(flops, world, ms_step)
 
-    single = len(runs) == 1 and runs[0].sh.n_hist > 0
+    single = len(runs) == 1 and runs[0].sh.n_hist > 0 and runs[0].kc == 0
     inc = incremental_compression(lf, runs[0], args, stream, cap, ev, flush_l2, g_att) \
         if single else None
     abl = ablation_1d(lf, runs[0], args, stream, cap, ev, flush_l2) if single else None
@@ -521,7 +561,8 @@ def run_lf(args, rank, world, local_rank):
         line["roofline_selection"] = {
             "bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": sel_gbs / pk["hbm_gbs"],
-            "kernels": "pool_blocks + block_scores + select_pick (lf_select_chunk)",
+            "kernels": "lf_select_chunk: select_stream_kernel (pooling, scores and picks in one "
+                       "launch) where the shape allows it",
             "peak_source": f"{src} hbm_gbs"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, dt, cores, n = oracle_sample(chunks, budget_s=10.0)

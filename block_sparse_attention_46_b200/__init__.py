@@ -21,7 +21,8 @@ __all__ = [
     "lf_select_chunk", "lf_select_workspace_size", "lf_block_sparse_attn_noalloc",
     "lf_noalloc_scratch_bytes", "lf_pooled_cache_bytes", "lf_pool_frames",
     "lf_select_chunk_cached", "lf_cag_schedule", "lf_select_chunk_1d",
-    "lf_status_string", "lf_abi_version", "lf_debug_configure", "derived", "LIB_PATH",
+    "lf_status_string", "lf_abi_version", "lf_debug_configure", "lf_select_current",
+    "derived", "current_blocks", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblf.so")
@@ -40,7 +41,8 @@ class LfShape(ctypes.Structure):
                 ("tokens_per_frame", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("n_cur_frames", ctypes.c_int32), ("n_hist", ctypes.c_int32),
                 ("n_sink", ctypes.c_int32), ("n_slots", ctypes.c_int32),
-                ("k_f", ctypes.c_int32), ("k_b", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("k_f", ctypes.c_int32), ("k_b", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("k_c", ctypes.c_int32)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -55,12 +57,13 @@ _SIGS = {
     "lf_select_blocks": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _P]),
     "lf_attn_workspace_size": (_SZ, [_SHP]),
     "lf_block_sparse_attn": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P, _P,
-                                            _P, _P, _SZ, _P]),
+                                            _P, _P, _P, _SZ, _P]),
+    "lf_select_current": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _SZ, _P]),
     "lf_forward_workspace_size": (_SZ, [_SHP]),
     "lf_select_workspace_size": (_SZ, [_SHP]),
     "lf_select_chunk": (ctypes.c_int, [_SHP, _P, _P, _I32P, _P, _P, _SZ, _P]),
     "lf_forward_chunk": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _I32P, _I32P, _P, _SZ, _P,
-                                        _P, _P, _P]),
+                                        _P, _P, _P, _P]),
     "lf_device_status": (ctypes.c_int, [ctypes.c_int]),
     "lf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "lf_abi_version": (ctypes.c_int, []),
@@ -96,7 +99,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 def make_shape(s) -> LfShape:
     """lf_shape from any object with the plain size fields (H, d, T, block, ...)."""
     return LfShape(s.H, s.d, s.T, s.block, s.n_cur_frames, s.n_hist, s.n_sink, s.n_slots,
-                   s.k_f, s.k_b, s.scale)
+                   s.k_f, s.k_b, s.scale, getattr(s, "k_c", 0))
 
 
 def derived(s):
@@ -105,6 +108,13 @@ def derived(s):
     kf = min(s.k_f, s.n_hist) if s.n_hist > 0 else 0
     kb = min(s.k_b, nbpf) if s.n_hist > 0 else 0
     return nbpf, s.n_cur_frames * nbpf, kf, kb
+
+
+def current_blocks(s) -> int:
+    """kc, the current-chunk blocks kept per query block (0: the dense current chunk)."""
+    nqb = s.n_cur_frames * -(-s.T // s.block)
+    k_c = getattr(s, "k_c", 0)
+    return min(k_c, nqb) if k_c > 0 else 0
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -199,6 +209,18 @@ def lf_select_chunk_1d(shape, q, k_cache, hist_slots, block_idx, workspace=None,
                                      _stream(stream)), "lf_select_chunk_1d")
 
 
+def lf_select_current(shape, q, k_cur, cur_idx, workspace=None, stream=None):
+    """Current-chunk block choice (shape.k_c >= 1): each query block's own block plus the
+    k_c - 1 best-scoring other current blocks, into cur_idx [H, n_qb, kc]."""
+    sh = make_shape(shape)
+    if workspace is None:
+        workspace = torch.empty(max(lf_forward_workspace_size(shape), 256), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().lf_select_current(ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(cur_idx),
+                                    _ptr(workspace), workspace.numel(), _stream(stream)),
+           "lf_select_current")
+
+
 def lf_pooled_cache_bytes(shape) -> int:
     sh = make_shape(shape)
     return int(load().lf_pooled_cache_bytes(ctypes.byref(sh)))
@@ -256,7 +278,7 @@ def lf_forward_workspace_size(shape) -> int:
 
 
 def lf_block_sparse_attn(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
-                         block_idx, out, lse=None, workspace=None, stream=None):
+                         block_idx, out, lse=None, workspace=None, stream=None, cur_idx=None):
     sh = make_shape(shape)
     hs, _k1 = _slots(hist_slots)
     ss, _k2 = _slots(sink_slots)
@@ -265,7 +287,7 @@ def lf_block_sparse_attn(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, s
                                 device=q.device)
     _check(load().lf_block_sparse_attn(
         ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_cache), _ptr(v_cache), hs, ss,
-        _ptr(block_idx), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _ptr(block_idx), _ptr(cur_idx), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)), "lf_block_sparse_attn")
 
 
@@ -287,7 +309,8 @@ def lf_block_sparse_attn_noalloc(shape, q, k_cur, v_cur, k_cache, v_cache, hist_
 
 
 def lf_forward_chunk(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
-                     out, lse=None, block_idx_out=None, workspace=None, stream=None):
+                     out, lse=None, block_idx_out=None, workspace=None, stream=None,
+                     cur_idx_out=None):
     sh = make_shape(shape)
     hs, _k1 = _slots(hist_slots)
     ss, _k2 = _slots(sink_slots)
@@ -297,4 +320,4 @@ def lf_forward_chunk(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_
     _check(load().lf_forward_chunk(
         ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_cache), _ptr(v_cache), hs, ss,
         _ptr(workspace), workspace.numel(), _ptr(out), _ptr(lse), _ptr(block_idx_out),
-        _stream(stream)), "lf_forward_chunk")
+        _ptr(cur_idx_out), _stream(stream)), "lf_forward_chunk")

@@ -34,6 +34,7 @@ int make_dims(const lf_shape* s, Dims* D) {
   if (s->n_hist + s->n_sink > LF_MAX_FRAMES) return LF_ERR_UNSUPPORTED;
   if ((s->n_hist > 0 || s->n_sink > 0) && s->n_slots < 1) return LF_ERR_INVALID_ARG;
   if (s->n_hist > 0 && (s->k_f < 1 || s->k_b < 1)) return LF_ERR_INVALID_ARG;
+  if (s->k_c < 0) return LF_ERR_INVALID_ARG;
   if (!(s->scale > 0.f) || s->scale > 1e30f) return LF_ERR_INVALID_ARG;
   const long long ncur = (long long)s->n_cur_frames * s->tokens_per_frame;
   if (ncur > (1LL << 30) / ((long long)s->H * s->d)) return LF_ERR_UNSUPPORTED;
@@ -48,8 +49,10 @@ int make_dims(const lf_shape* s, Dims* D) {
   d.kf = d.F > 0 ? (s->k_f < d.F ? s->k_f : d.F) : 0;
   d.kb = d.F > 0 ? (s->k_b < d.nbpf ? s->k_b : d.nbpf) : 0;
   d.nsel = d.kf * d.kb;
+  d.kc = s->k_c > 0 ? (s->k_c < d.nqb ? s->k_c : d.nqb) : 0;
   d.scale = s->scale;
   if (d.nsel > LF_MAX_SELECTED) return LF_ERR_UNSUPPORTED;
+  if (d.kc > 0 && d.nqb > LF_MAX_CUR_BLOCKS) return LF_ERR_UNSUPPORTED;
   if (lf::plan_stride(d) > lf::kMaxPlan) return LF_ERR_UNSUPPORTED;
   *D = d;
   return LF_OK;
@@ -101,16 +104,21 @@ int encode_rows(CUtensorMap* m, const void* base, int HD, long long rows, int sl
 }
 
 // ---------------------------------------------------------------- launches
+// Pooling of the query blocks, the history key blocks (D.F frames) and, when kc_blk is
+// given, the current chunk's key blocks; then (k_frm given) the history frame means.
 int launch_compress(const Dims& D, const void* q, const void* k_cache, const int32_t* hist_slots,
-                    float* q_blk, float* k_blk, float* k_frm, cudaStream_t st) {
+                    float* q_blk, float* k_blk, float* k_frm, cudaStream_t st,
+                    const void* k_cur = nullptr, float* kc_blk = nullptr) {
   lf::PoolArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   a.q_blk = q_blk;
   a.k_blk = k_blk;
   a.k_pool = nullptr;
+  a.k_cur = static_cast<const __nv_bfloat16*>(k_cur);
+  a.kc_blk = kc_blk;
   for (int f = 0; f < D.F; ++f) a.hist_slots[f] = hist_slots[f];
-  const int units = D.nqb + D.F * D.nbpf;
+  const int units = D.nqb + D.F * D.nbpf + (kc_blk != nullptr ? D.nqb : 0);
   const int vecs = D.H * D.d / 8;
   dim3 grid(units, lf::cdiv(vecs, lf::kPoolCols));
   lf::pool_blocks_kernel<<<grid, lf::kPoolThreads, 0, st>>>(a, D);
@@ -145,6 +153,19 @@ int launch_select_frames(const Dims& D, const float* q_blk, const float* k_frm,
   if (e != cudaSuccess) return LF_ERR_CUDA;
   dim3 grid(lf::cdiv(D.nqb, lf::kSelWarps), D.H);
   kern<<<grid, lf::kSelWarps * 32, smem, st>>>(q_blk, k_frm, frame_idx, frame_score, D);
+  return cuda_status(cudaGetLastError());
+}
+
+// Current-chunk block choice: own block plus the kc - 1 best others, per (head, query block).
+int launch_select_current(const Dims& D, const float* q_blk, const float* kc_blk,
+                          int32_t* cur_idx, cudaStream_t st) {
+  const size_t smem = ((size_t)D.nqb * (D.d + 4) + (size_t)lf::kSelWarps * D.d) * sizeof(float);
+  if (smem > kMaxSmem) return LF_ERR_UNSUPPORTED;
+  auto kern = D.d == 128 ? lf::select_current_kernel<128> : lf::select_current_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return LF_ERR_CUDA;
+  dim3 grid(lf::cdiv(D.nqb, lf::kSelWarps), D.H);
+  kern<<<grid, lf::kSelWarps * 32, smem, st>>>(q_blk, kc_blk, cur_idx, D);
   return cuda_status(cudaGetLastError());
 }
 
@@ -190,8 +211,8 @@ Split make_split(const Dims& D, int n_sm) {
   if (R == 0 || 2 * R > n_sm) return sp;
   int p = n_sm / R;
   p = p < lf::kMaxPieces ? p : lf::kMaxPieces;
-  const int n_dense = lf::cdiv(D.ncur, 128);      // every tile has at least this many
-  p = p < n_dense ? p : n_dense;
+  const int n_min = lf::min_key_tiles(D);        // every tile has at least this many
+  p = p < n_min ? p : n_min;
   if (p < 2) return sp;
   sp.n_whole = ntot - R;
   sp.n_tail = R;
@@ -243,15 +264,16 @@ int launch_attn_t(const Dims& D, lf::AttnParams& p, int grid, cudaStream_t st) {
 
 int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_cur,
                 const void* k_cache, const void* v_cache, const int32_t* hist_slots,
-                const int32_t* sink_slots, const int32_t* block_idx, void* out, float* lse,
-                void* workspace, cudaStream_t st, bool plans_ready = false) {
+                const int32_t* sink_slots, const int32_t* block_idx, const int32_t* cur_idx,
+                void* out, float* lse, void* workspace, cudaStream_t st,
+                bool plans_ready = false) {
   const int n_sm = sm_count();
   if (n_sm <= 0) return LF_ERR_CUDA;
   const AttnWs w = carve_attn(D, workspace, n_sm);
   // key plans (unless the fused selection already wrote them), then the launch order
   if (!plans_ready)
     lf::plan_kernel<<<dim3(lf::cdiv(lf::tile_count(D), lf::kPlanWarps), D.H), lf::kPlanWarps * 32, 0, st>>>(
-        D.F > 0 ? block_idx : nullptr, w.plan, w.plan_cnt, D);
+        D.F > 0 ? block_idx : nullptr, D.kc > 0 ? cur_idx : nullptr, w.plan, w.plan_cnt, D);
   const Split sp = make_split(D, n_sm);
   lf::schedule_kernel<<<1, 1024, 0, st>>>(w.plan_cnt, w.order, D,
                                           sp.n_tail > 0 ? sp.n_whole : lf::tile_count(D) * D.H);
@@ -297,8 +319,8 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
 
 // forward workspace carve-up
 struct FwdWs {
-  float *q_blk, *k_blk, *k_frm, *scores;
-  int32_t *frame_idx, *block_idx;
+  float *q_blk, *k_blk, *k_frm, *scores, *kc_blk;
+  int32_t *frame_idx, *block_idx, *cur_idx, *sync;
   void* attn;
   size_t bytes;
 };
@@ -314,6 +336,9 @@ FwdWs carve(const Dims& D, void* base) {
   w.scores = reinterpret_cast<float*>(take((size_t)D.H * D.nqb * D.F * D.nbpf * 4));
   w.frame_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.kf * 4));
   w.block_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.nsel * 4));
+  w.kc_blk = reinterpret_cast<float*>(take((size_t)D.H * (D.kc > 0 ? D.nqb : 0) * D.d * 4));
+  w.cur_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.kc * 4));
+  w.sync = reinterpret_cast<int32_t*>(take((size_t)(1 + 2 * D.H) * 4));
   w.attn = take(attn_ws_bytes(D));
   w.bytes = off;
   return w;
@@ -349,33 +374,96 @@ int launch_scores_pick(const Dims& D, const FwdWs& w, const float* k_pool,
   if (cudaFuncSetAttribute(lf::select_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return LF_ERR_CUDA;
+  // with a sparse current chunk the key plans also hold current blocks: plan_kernel
+  // builds them, the pick kernel writes the lists only
   lf::select_pick_kernel<<<dim3(lf::cdiv(D.nqb, lf::kFuseQb), D.H), lf::kPickThreads, smem,
-                           stream>>>(w.scores, bidx, aw.plan, aw.plan_cnt, D);
+                           stream>>>(w.scores, bidx, D.kc > 0 ? nullptr : aw.plan, aw.plan_cnt, D);
   return cuda_status(cudaGetLastError());
 }
 
-// Stages (a)-(c) into `bidx`: pooling, then the fused selection (which also writes the
-// attention key plans into the workspace) when the shape allows it, else the separate
-// frame-pooling, frame-selection and block-selection kernels.
+// Whether stages (a)-(c) run as the single-launch selection kernel.
+bool stream_ok(const Dims& D) {
+  if (D.kc > 0 || !lf::fused_select_ok(D)) return false;
+  const size_t smem = D.d == 128 ? lf::stream_smem<128>(D) : lf::stream_smem<64>(D);
+  return smem <= kMaxSmem;
+}
+
+// Stages (a)-(c) in one launch (lf::select_stream_kernel): the work counters are zeroed,
+// then every pooling, scoring and pick unit runs in ticket order.
+int launch_stream(const Dims& D, const void* q, const void* k_cache, const int32_t* hist_slots,
+                  const FwdWs& w, const AttnWs& aw, int32_t* bidx, cudaStream_t stream) {
+  if (cudaMemsetAsync(w.sync, 0, (size_t)(1 + 2 * D.H) * sizeof(int32_t), stream) != cudaSuccess)
+    return LF_ERR_CUDA;
+  lf::StreamArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  a.q_blk = w.q_blk;
+  a.scores = w.scores;
+  a.block_idx = bidx;
+  a.plan = aw.plan;
+  a.plan_cnt = aw.plan_cnt;
+  a.sync = w.sync;
+  a.wait_limit_ns = g_dbg_wait_limit_ns;
+  for (int f = 0; f < D.F; ++f) a.hist_slots[f] = hist_slots[f];
+  const int np = lf::stream_parts(D);
+  const int units = D.H * (D.Fc + D.F) * np + D.H * lf::cdiv(D.nqb, lf::kFuseQb);
+  auto kern = D.d == 128 ? lf::select_stream_kernel<128> : lf::select_stream_kernel<64>;
+  const size_t smem = D.d == 128 ? lf::stream_smem<128>(D) : lf::stream_smem<64>(D);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LF_ERR_CUDA;
+  kern<<<units, lf::kStreamThreads, smem, stream>>>(a, D);
+  return cuda_status(cudaGetLastError());
+}
+
+// Stages (a)-(c) into `bidx`: the single-launch selection when the shape allows it, else
+// pooling and the pick kernel, else the separate frame-pooling, frame-selection and
+// block-selection kernels.  The first two also write the attention key plans into the
+// workspace (*plans_ready).
 int run_select(const Dims& D, const void* q, const void* k_cache, const int32_t* hist_slots,
-               const FwdWs& w, int32_t* bidx, cudaStream_t stream, bool* plans_ready) {
+               const FwdWs& w, int32_t* bidx, cudaStream_t stream, bool* plans_ready,
+               const void* k_cur = nullptr) {
   int rc;
   *plans_ready = false;
+  float* kc_blk = k_cur != nullptr ? w.kc_blk : nullptr;   // also pool the current keys
+  if (k_cur == nullptr && stream_ok(D)) {
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return LF_ERR_CUDA;
+    if ((rc = launch_stream(D, q, k_cache, hist_slots, w, carve_attn(D, w.attn, n_sm), bidx,
+                            stream)) != LF_OK)
+      return rc;
+    *plans_ready = true;
+    return LF_OK;
+  }
   if (lf::fused_select_ok(D) && lf::fused_select_smem(D) <= kMaxSmem) {
-    if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, nullptr, stream)) != LF_OK)
+    if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, nullptr, stream,
+                              k_cur, kc_blk)) != LF_OK)
       return rc;
     const int n_sm = sm_count();
     if (n_sm <= 0) return LF_ERR_CUDA;
     const AttnWs aw = carve_attn(D, w.attn, n_sm);
     if ((rc = launch_scores_pick(D, w, nullptr, hist_slots, aw, bidx, stream)) != LF_OK) return rc;
-    *plans_ready = true;
+    *plans_ready = D.kc == 0;
     return LF_OK;
   }
-  if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, w.k_frm, stream)) != LF_OK)
+  if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, w.k_frm, stream,
+                            k_cur, kc_blk)) != LF_OK)
     return rc;
   if ((rc = launch_select_frames(D, w.q_blk, w.k_frm, w.frame_idx, nullptr, stream)) != LF_OK)
     return rc;
   return launch_select_blocks(D, w.q_blk, w.k_blk, w.frame_idx, bidx, nullptr, stream);
+}
+
+// Current-chunk selection: pooling of the query and current key blocks (one launch),
+// then the own block plus the kc - 1 best others per (head, query block).
+int run_select_current(const Dims& D, const void* q, const void* k_cur, const FwdWs& w,
+                       int32_t* cur_idx, cudaStream_t stream) {
+  Dims Dq = D;
+  Dq.F = 0;                                      // no history units in this pooling launch
+  int rc = launch_compress(Dq, q, nullptr, nullptr, w.q_blk, nullptr, nullptr, stream, k_cur,
+                           w.kc_blk);
+  if (rc != LF_OK) return rc;
+  return launch_select_current(D, w.q_blk, w.kc_blk, cur_idx, stream);
 }
 
 // ---------------------------------------------------------------- fixed scratch
@@ -554,8 +642,9 @@ size_t lf_attn_workspace_size(const lf_shape* shape) {
 int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur,
                          const void* v_cur, const void* k_cache, const void* v_cache,
                          const int32_t* hist_slots, const int32_t* sink_slots,
-                         const int32_t* block_idx, void* out, float* lse,
-                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                         const int32_t* block_idx, const int32_t* cur_idx, void* out,
+                         float* lse, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
   Dims D;
   int rc = make_dims(shape, &D);
   if (rc != LF_OK) return rc;
@@ -567,6 +656,7 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
                         !aligned(v_cache, 16)))
     return LF_ERR_INVALID_ARG;
   if (D.F > 0 && (block_idx == nullptr || !aligned(block_idx, 4))) return LF_ERR_INVALID_ARG;
+  if (D.kc > 0 && (cur_idx == nullptr || !aligned(cur_idx, 4))) return LF_ERR_INVALID_ARG;
   if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
   if ((rc = check_slots(sink_slots, D.S, D.n_slots)) != LF_OK) return rc;
   const size_t need = attn_ws_bytes(D);
@@ -574,7 +664,7 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need)
     return LF_ERR_WORKSPACE;
   return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, block_idx,
-                     out, lse, workspace, stream);
+                     cur_idx, out, lse, workspace, stream);
 }
 
 size_t lf_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
@@ -587,13 +677,15 @@ int lf_block_sparse_attn_noalloc(const lf_shape* shape, const void* q, const voi
   Dims D;
   int rc = make_dims(shape, &D);
   if (rc != LF_OK) return rc;
+  if (D.kc > 0) return LF_ERR_INVALID_ARG;                     // takes no current-chunk list
   const size_t need = attn_ws_bytes(D);
   if (need == 0) return LF_ERR_CUDA;
   if (need > kNoAllocScratchBytes) return LF_ERR_WORKSPACE;   // shape needs more scratch
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch)) != LF_OK) return rc;
   return lf_block_sparse_attn(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots,
-                              block_idx, out, lse, scratch, kNoAllocScratchBytes, stream);
+                              block_idx, nullptr, out, lse, scratch, kNoAllocScratchBytes,
+                              stream);
 }
 
 size_t lf_forward_workspace_size(const lf_shape* shape) {
@@ -606,13 +698,14 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
                      const void* v_cur, const void* k_cache, const void* v_cache,
                      const int32_t* hist_slots, const int32_t* sink_slots,
                      void* workspace, size_t workspace_bytes, void* out, float* lse,
-                     int32_t* block_idx_out, cudaStream_t stream) {
+                     int32_t* block_idx_out, int32_t* cur_idx_out, cudaStream_t stream) {
   Dims D;
   int rc = make_dims(shape, &D);
   if (rc != LF_OK) return rc;
   if (q == nullptr || k_cur == nullptr || v_cur == nullptr || out == nullptr ||
       !aligned(q, 16) || !aligned(k_cur, 16) || !aligned(v_cur, 16) || !aligned(out, 16) ||
-      (lse && !aligned(lse, 4)) || (block_idx_out && !aligned(block_idx_out, 4)))
+      (lse && !aligned(lse, 4)) || (block_idx_out && !aligned(block_idx_out, 4)) ||
+      (cur_idx_out && !aligned(cur_idx_out, 4)))
     return LF_ERR_INVALID_ARG;
   if (D.F + D.S > 0 && (k_cache == nullptr || v_cache == nullptr || !aligned(k_cache, 16) ||
                         !aligned(v_cache, 16)))
@@ -624,11 +717,36 @@ int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
     return LF_ERR_WORKSPACE;
   const FwdWs w = carve(D, workspace);
   int32_t* bidx = block_idx_out ? block_idx_out : w.block_idx;
+  int32_t* cidx = cur_idx_out ? cur_idx_out : w.cur_idx;
   bool plans_ready = false;
-  if (D.F > 0 && (rc = run_select(D, q, k_cache, hist_slots, w, bidx, stream, &plans_ready)) != LF_OK)
-    return rc;
-  return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, bidx, out,
-                     lse, w.attn, stream, plans_ready);
+  if (D.F > 0) {
+    // with a sparse current chunk the same pooling launch also pools the current keys
+    if ((rc = run_select(D, q, k_cache, hist_slots, w, bidx, stream, &plans_ready,
+                         D.kc > 0 ? k_cur : nullptr)) != LF_OK)
+      return rc;
+    if (D.kc > 0 && (rc = launch_select_current(D, w.q_blk, w.kc_blk, cidx, stream)) != LF_OK)
+      return rc;
+  } else if (D.kc > 0) {
+    if ((rc = run_select_current(D, q, k_cur, w, cidx, stream)) != LF_OK) return rc;
+  }
+  return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, bidx, cidx,
+                     out, lse, w.attn, stream, plans_ready);
+}
+
+int lf_select_current(const lf_shape* shape, const void* q, const void* k_cur,
+                      int32_t* cur_idx, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (D.kc < 1) return LF_ERR_INVALID_ARG;
+  if (q == nullptr || k_cur == nullptr || cur_idx == nullptr || !aligned(q, 16) ||
+      !aligned(k_cur, 16) || !aligned(cur_idx, 4))
+    return LF_ERR_INVALID_ARG;
+  const FwdWs need = carve(D, nullptr);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need.bytes)
+    return LF_ERR_WORKSPACE;
+  return run_select_current(D, q, k_cur, carve(D, workspace), cur_idx, stream);
 }
 
 size_t lf_select_workspace_size(const lf_shape* shape) { return lf_forward_workspace_size(shape); }

@@ -34,7 +34,8 @@ constexpr int kAttnThreads = 384;
 
 // Plan entry: bits 0-1 = which of the tile's two query blocks selected it (bit 0: rows
 // 0-63 or the single 128-row block; bit 1: rows 64-127), bits 4-15 = block in frame,
-// bits 16-27 = frame position (sinks first, then history frames).
+// bits 16-27 = frame position: sinks [0, S), history frames [S, S + F), and, when the
+// current chunk is sparse, the current chunk's frames [S + F, S + F + F_c).
 __host__ __device__ inline uint32_t plan_pack(int p, int b, uint32_t mask) {
   return ((uint32_t)p << 16) | ((uint32_t)b << 4) | mask;
 }
@@ -43,7 +44,13 @@ __host__ __device__ inline int tile_count(const Dims& D) {
   return D.B == 64 ? cdiv(D.nqb, 2) : D.nqb;
 }
 __host__ __device__ inline int plan_stride(const Dims& D) {
-  return D.S * D.nbpf + (D.B == 64 ? 2 : 1) * D.nsel;
+  return D.S * D.nbpf + (D.B == 64 ? 2 : 1) * (D.kc + D.nsel);
+}
+// Key tiles every query tile has at least: the dense current chunk, or the key blocks of
+// one query block's lists (sinks, kept current blocks, selected history blocks).
+__host__ __device__ inline int min_key_tiles(const Dims& D) {
+  const int per = D.B == 64 ? 2 : 1;
+  return (D.kc > 0 ? 0 : cdiv(D.ncur, 128)) + cdiv(D.S * D.nbpf + D.kc + D.nsel, per);
 }
 
 // ---------------------------------------------------------------------------------
@@ -61,14 +68,15 @@ __device__ __forceinline__ int lower_bound_s(const int32_t* a, int n, int v) {
   return lo;
 }
 
-// One warp writes a tile's key plan from its query blocks' ascending block lists A and
-// B (shared memory, already validated; nB = 0 when the tile has one query block): sink
-// blocks first, then the sorted union.  Returns the entry count.
-__device__ __forceinline__ int warp_write_plan(const int32_t* sa, int nA, const int32_t* sb,
-                                               int nB, uint32_t* out, const Dims& D) {
+// One warp writes the sorted union of a tile's two ascending id lists A and B (shared
+// memory, already validated; nB = 0 when the tile has one query block) at out[0..), each
+// id as the plan entry of frame position p_base + id / nbpf, block id % nbpf, with a bit
+// per list holding it.  The position of an element in the union is its rank in its own
+// list plus the number of smaller elements of the other list minus the common elements
+// counted twice.  Returns the entry count.
+__device__ __forceinline__ int warp_write_union(const int32_t* sa, int nA, const int32_t* sb,
+                                                int nB, uint32_t* out, int p_base, int nbpf) {
   const int lane = threadIdx.x & 31;
-  const int nsink = D.S * D.nbpf;
-  for (int e = lane; e < nsink; e += 32) out[e] = plan_pack(e / D.nbpf, e % D.nbpf, 3u);
   const uint32_t lt = (1u << lane) - 1u;
   int carry = 0;
   for (int i0 = 0; i0 < nA; i0 += 32) {
@@ -80,7 +88,7 @@ __device__ __forceinline__ int warp_write_plan(const int32_t* sa, int nA, const 
     const uint32_t bal = __ballot_sync(0xffffffffu, inB);
     if (valid) {
       const int pos = i + cb - (carry + __popc(bal & lt));
-      out[nsink + pos] = plan_pack(D.S + a / D.nbpf, a % D.nbpf, inB ? 3u : 1u);
+      out[pos] = plan_pack(p_base + a / nbpf, a % nbpf, inB ? 3u : 1u);
     }
     carry += __popc(bal);
   }
@@ -95,18 +103,39 @@ __device__ __forceinline__ int warp_write_plan(const int32_t* sa, int nA, const 
     const uint32_t bal = __ballot_sync(0xffffffffu, inA);
     if (valid && !inA) {
       const int pos = j + ca - (carry + __popc(bal & lt));
-      out[nsink + pos] = plan_pack(D.S + b / D.nbpf, b % D.nbpf, 2u);
+      out[pos] = plan_pack(p_base + b / nbpf, b % nbpf, 2u);
     }
     carry += __popc(bal);
   }
-  return nsink + nA + nB - ncommon;
+  return nA + nB - ncommon;
+}
+
+// Stages one query tile's two ascending lists of n ids each (B absent when qbB < 0) from
+// `lists` [H, nqb, n] into shared memory and checks them (ids in [0, lim), strictly
+// ascending).  Returns false, for the whole warp, if either list is invalid.
+__device__ __forceinline__ bool warp_stage_lists(const int32_t* lists, int n, int lim, int h,
+                                                 int qa, int qbB, const Dims& D, int32_t* sa,
+                                                 int32_t* sb) {
+  const int lane = threadIdx.x & 31;
+  stage_words(sa, lists + ((size_t)h * D.nqb + qa) * n, n, lane, 32);
+  if (qbB >= 0) stage_words(sb, lists + ((size_t)h * D.nqb + qbB) * n, n, lane, 32);
+  __syncwarp();
+  const int nB = qbB >= 0 ? n : 0;
+  bool bad = false;
+  for (int i = lane; i < n; i += 32) bad |= sa[i] < 0 || sa[i] >= lim || (i > 0 && sa[i - 1] >= sa[i]);
+  for (int i = lane; i < nB; i += 32) bad |= sb[i] < 0 || sb[i] >= lim || (i > 0 && sb[i - 1] >= sb[i]);
+  return !__any_sync(0xffffffffu, bad);
 }
 
 constexpr int kPlanWarps = 4;
 
+// Key plan of each (query tile, head), one warp: sink blocks (kept by both query blocks),
+// then the union of the query blocks' current-chunk lists (when the current chunk is
+// sparse), then the union of their history lists.  A list that fails validation is
+// dropped and LF_ERR_BAD_INDEX recorded.
 __global__ void __launch_bounds__(kPlanWarps * 32)
-plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
-            int32_t* __restrict__ plan_cnt, const Dims D) {
+plan_kernel(const int32_t* __restrict__ block_idx, const int32_t* __restrict__ cur_idx,
+            uint32_t* __restrict__ plan, int32_t* __restrict__ plan_cnt, const Dims D) {
   __shared__ int32_t s_ab[kPlanWarps][2][LF_MAX_SELECTED];
   const int ntiles = tile_count(D);
   const int t = blockIdx.x * kPlanWarps + (threadIdx.x >> 5), h = blockIdx.y;
@@ -115,30 +144,29 @@ plan_kernel(const int32_t* __restrict__ block_idx, uint32_t* __restrict__ plan,
   int32_t* sa = s_ab[threadIdx.x >> 5][0];
   int32_t* sb = s_ab[threadIdx.x >> 5][1];
   uint32_t* out = plan + ((size_t)h * ntiles + t) * plan_stride(D);
-  int nA = 0, nB = 0;
-  if (D.F > 0 && D.nsel > 0 && block_idx != nullptr) {
-    const int qa = D.B == 64 ? 2 * t : t;
-    const int qbB = (D.B == 64 && 2 * t + 1 < D.nqb) ? 2 * t + 1 : -1;
-    nA = D.nsel;
-    nB = qbB >= 0 ? D.nsel : 0;
-    const int32_t* A = block_idx + ((size_t)h * D.nqb + qa) * D.nsel;
-    const int32_t* B = qbB >= 0 ? block_idx + ((size_t)h * D.nqb + qbB) * D.nsel : nullptr;
-    const int lim = D.F * D.nbpf;
-    bool bad = false;
-    stage_words(sa, A, nA, lane, 32);
-    if (nB > 0) stage_words(sb, B, nB, lane, 32);
+  const int qa = D.B == 64 ? 2 * t : t;
+  const int qbB = (D.B == 64 && 2 * t + 1 < D.nqb) ? 2 * t + 1 : -1;
+  const int nsink = D.S * D.nbpf;
+  for (int e = lane; e < nsink; e += 32) out[e] = plan_pack(e / D.nbpf, e % D.nbpf, 3u);
+  int cnt = nsink;
+  bool bad = false;
+  if (D.kc > 0) {
+    if (warp_stage_lists(cur_idx, D.kc, D.nqb, h, qa, qbB, D, sa, sb))
+      cnt += warp_write_union(sa, D.kc, sb, qbB >= 0 ? D.kc : 0, out + cnt, D.S + D.F, D.nbpf);
+    else
+      bad = true;
     __syncwarp();
-    for (int i = lane; i < nA; i += 32)
-      bad |= sa[i] < 0 || sa[i] >= lim || (i > 0 && sa[i - 1] >= sa[i]);
-    for (int i = lane; i < nB; i += 32)
-      bad |= sb[i] < 0 || sb[i] >= lim || (i > 0 && sb[i - 1] >= sb[i]);
-    if (__any_sync(0xffffffffu, bad)) {       // the selected lists are dropped
-      if (lane == 0) record_status(LF_ERR_BAD_INDEX);
-      nA = nB = 0;
-    }
   }
-  const int cnt = warp_write_plan(sa, nA, sb, nB, out, D);
-  if (lane == 0) plan_cnt[(size_t)h * ntiles + t] = cnt;
+  if (D.F > 0 && D.nsel > 0 && block_idx != nullptr) {
+    if (warp_stage_lists(block_idx, D.nsel, D.F * D.nbpf, h, qa, qbB, D, sa, sb))
+      cnt += warp_write_union(sa, D.nsel, sb, qbB >= 0 ? D.nsel : 0, out + cnt, D.S, D.nbpf);
+    else
+      bad = true;
+  }
+  if (lane == 0) {
+    if (bad) record_status(LF_ERR_BAD_INDEX);
+    plan_cnt[(size_t)h * ntiles + t] = cnt;
+  }
 }
 
 // ---------------------------------------------------------------------------------
@@ -346,7 +374,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   const int tokB = qbB >= 0 ? (qbB / D.nbpf) * D.T + (qbB % D.nbpf) * BLK : D.ncur;
 
   const int cnt = P.plan_cnt[tile];
-  const int n_dense = cdiv(D.ncur, 128);
+  const int n_dense = D.kc > 0 ? 0 : cdiv(D.ncur, 128);   // sparse current chunk: in the plan
   const int n_sparse = BLK == 64 ? cdiv(cnt, 2) : cnt;
   const int n_tile = n_dense + n_sparse;
   // this CTA's key tiles: [j0, j0 + n_iter); local index l = j - j0 drives the pipeline
@@ -425,16 +453,27 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
                         h * HD + c * 64, row);
         } else {
           const int u = j - n_dense;
-          int slot_id = 0, tok = D.T;                   // default: all rows out of bounds
+          int slot_id = 0, tok = 0;
+          int p = -1;                                    // -1: padding past the plan's end
           const int e = BLK == 64 ? 2 * u + box : u;
           if (e < cnt) {
             const uint32_t pe = s_plan[e];
-            slot_id = P.slots[pe >> 16];
+            p = (int)(pe >> 16);
             tok = (int)((pe >> 4) & 0xFFFu) * BLK + (BLK == 64 ? 0 : box * 64);
+            if (p < D.S + D.F) slot_id = P.slots[p];
           }
-          for (int c = 0; c < L::NH; ++c)
-            tma_load_3d(st + c * L::kRegion + box * 64 * 128, tm_hist, &full[slot],
-                        h * HD + c * 64, tok, slot_id);
+          if (p < 0 || p >= D.S + D.F) {
+            // a block of the current chunk (2-D map), or padding: rows from ncur on are
+            // out of bounds and read as zero (the columns are masked anyway)
+            const int row = p < 0 ? D.ncur : (p - D.S - D.F) * D.T + tok;
+            for (int c = 0; c < L::NH; ++c)
+              tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
+                          h * HD + c * 64, row);
+          } else {
+            for (int c = 0; c < L::NH; ++c)
+              tma_load_3d(st + c * L::kRegion + box * 64 * 128, tm_hist, &full[slot],
+                          h * HD + c * 64, tok, slot_id);
+          }
         }
       }
     }
@@ -477,7 +516,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       return true;
     };
     bool ok = mbar_wait(&bars[kBarQ], 0, s_abort, P.wait_limit_ns);
-    if (ok) ok = issue_s(0);
+    if (ok && n_iter > 0) ok = issue_s(0);
     if (ok && n_iter > 1) ok = issue_s(1);
     for (int l = 0; ok && l < n_iter; ++l) {
       const int s = l & 1;

@@ -18,6 +18,7 @@ struct Dims {
   int nqb;             // query blocks, Fc * nbpf
   int ncur;            // current-chunk tokens, Fc * T
   int nsel;            // selected blocks per query block, kf * kb
+  int kc;              // current-chunk blocks kept per query block; 0: dense current chunk
   float scale;
 };
 

@@ -138,20 +138,25 @@ block_scores_kernel(const __grid_constant__ ScoreArgs a, const Dims D) {
 constexpr int kPickThreads = 256;
 constexpr int kFuseWords = kFuseMaxBlocks / 32;
 
-__global__ void __launch_bounds__(kPickThreads)
-select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block_idx,
-                   uint32_t* __restrict__ plan, int32_t* __restrict__ plan_cnt, const Dims D) {
-  extern __shared__ float4 sm4[];
+// The pick of one group of kFuseQb query blocks of head h (qb0 = first), by a whole CTA of
+// kPickThreads threads; `sm` is dynamic shared memory of at least fused_select_smem(D)
+// bytes.  Score rows are read with L2-coherent loads (they may have been written by other
+// CTAs of the same launch).  plan == nullptr: the lists only.
+__device__ __forceinline__ void pick_group(const float* __restrict__ scores,
+                                           int32_t* __restrict__ block_idx,
+                                           uint32_t* __restrict__ plan,
+                                           int32_t* __restrict__ plan_cnt, const Dims& D, int h,
+                                           int qb0, float* sm) {
   const int NB = D.F * D.nbpf;
-  float* sc = reinterpret_cast<float*>(sm4);                        // [kFuseQb][NB]
+  float* sc = sm;                                                   // [kFuseQb][NB]
   int32_t* sl = reinterpret_cast<int32_t*>(sc + (size_t)kFuseQb * NB);   // [kFuseQb][nsel]
   int32_t* sf = sl + kFuseQb * D.nsel;                              // [kFuseQb][kf]
-  const int h = blockIdx.y, qb0 = blockIdx.x * kFuseQb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   {
     // the group's rows of the score matrix are contiguous: [qb0, qb0 + kFuseQb) x NB
     const int ng = min(kFuseQb, D.nqb - qb0);
-    stage_words(sc, scores + ((size_t)h * D.nqb + qb0) * NB, ng * NB, threadIdx.x, blockDim.x);
+    const float* src = scores + ((size_t)h * D.nqb + qb0) * NB;
+    for (int i = threadIdx.x; i < ng * NB; i += blockDim.x) sc[i] = __ldcg(src + i);
   }
   __syncthreads();
 
@@ -198,6 +203,7 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
     const int g = i / D.nsel, qb = qb0 + g;
     if (qb < D.nqb) block_idx[((size_t)h * D.nqb + qb) * D.nsel + i % D.nsel] = sl[i];
   }
+  if (plan == nullptr) return;                             // lists only
 
   // key plans of the group's tiles
   __shared__ uint32_t s_bits[2][kFuseWords];   // blocks chosen by the tile's query blocks
@@ -247,6 +253,229 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
       }
     }
     __syncthreads();                                       // the bitmaps are reused
+  }
+}
+
+// Per (head, group of kFuseQb query blocks): frame scores by linearity from the block
+// scores, frame top-k, block top-k in each chosen frame, block_idx, and the key plans of
+// the group's query tiles.  A tile's plan is written by the whole CTA from two bitmaps
+// over the F * n_bpf history blocks (one per query block of the tile): the union's bits
+// in id order give the entries, a prefix count of the union's words their positions.
+__global__ void __launch_bounds__(kPickThreads)
+select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block_idx,
+                   uint32_t* __restrict__ plan, int32_t* __restrict__ plan_cnt, const Dims D) {
+  extern __shared__ float4 sm4[];
+  pick_group(scores, block_idx, plan, plan_cnt, D, blockIdx.y, blockIdx.x * kFuseQb,
+             reinterpret_cast<float*>(sm4));
+}
+
+// ---------------------------------------------------------------------------------
+// Stages (a)-(c) in one launch.  Work units are handed out in order by an atomic ticket:
+//   [0, UQ)            pooling of the query blocks of (head, current frame, part),
+//   [UQ, UQ + UH)      pooling of the key blocks of (head, history frame, part) and their
+//                      scores against every pooled query block of the head,
+//   [UQ + UH, total)   the pick of (head, group of kFuseQb query blocks).
+// A part is a run of at most kStreamBlocks consecutive blocks of one frame, one head's d
+// channels.  A history unit waits until its head's query units are done, a pick unit until
+// its head's history units are done; the units waited for hold lower tickets, so they were
+// taken by CTAs that already run, and every wait ends (each is also bounded in time).
+// Sums are in the order of pool_blocks_kernel (four runs of a block's tokens, each in token
+// order, then the runs in order, times the reciprocal of the length) and of
+// block_scores_kernel (one fma chain over the channels in order), so pooled values, scores,
+// lists and plans are bit-identical to the three-kernel path.
+// ---------------------------------------------------------------------------------
+constexpr int kStreamThreads = 256;
+constexpr int kStreamBlocks = 16;          // blocks per pooling part, at most
+
+struct StreamArgs {
+  const __nv_bfloat16* q;        // [ncur, H, d]
+  const __nv_bfloat16* k_cache;  // [n_slots, T, H, d]
+  float* q_blk;                  // [H, nqb, d]
+  float* scores;                 // [H, nqb, F * nbpf]
+  int32_t* block_idx;            // [H, nqb, nsel]
+  uint32_t* plan;                // key plans, or null (lists only)
+  int32_t* plan_cnt;
+  int32_t* sync;                 // [1 + 2H], zero at launch: ticket, q_done[H], hist_done[H]
+  uint64_t wait_limit_ns;
+  int hist_slots[LF_MAX_FRAMES];
+};
+
+__host__ __device__ inline int stream_parts(const Dims& D) { return cdiv(D.nbpf, kStreamBlocks); }
+
+template <int HD>
+__host__ __device__ inline size_t stream_smem(const Dims& D) {
+  constexpr int VPR = HD / 8, BB = kStreamThreads / (4 * VPR);
+  const size_t pool = (size_t)BB * 4 * HD * 4 + (size_t)kStreamBlocks * (HD + 4) * 4 +
+                      (size_t)D.nqb * (HD + 4) * 4;
+  const size_t pick = fused_select_smem(D);
+  return pool > pick ? pool : pick;
+}
+
+// Waits (thread 0, then the whole CTA) until *counter reaches target; false on timeout.
+__device__ __forceinline__ bool cta_wait_count(const int32_t* counter, int target,
+                                               uint64_t limit_ns) {
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    if (*reinterpret_cast<const volatile int32_t*>(counter) < target) {
+      const uint64_t t0 = globaltimer_ns();
+      while (*reinterpret_cast<const volatile int32_t*>(counter) < target) {
+        if (globaltimer_ns() - t0 > limit_ns) {
+          record_status(LF_ERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// Publishes this CTA's global writes, then adds one to *counter.
+__device__ __forceinline__ void cta_signal(int32_t* counter) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAdd(counter, 1);
+}
+
+// Pools blocks [b0, b1) of one frame for head h (frame = token 0 of the frame, row pitch
+// H*d bf16) and hands each block mean to out(b, channel, value).  Batches of BB blocks:
+// thread (block bi, run g, vector c) sums its run of the block's tokens in token order.
+template <int HD, typename Out>
+__device__ __forceinline__ void pool_part(const __nv_bfloat16* __restrict__ frame, int h,
+                                          int b0, int b1, const Dims& D, float* part, Out out) {
+  constexpr int VPR = HD / 8, BB = kStreamThreads / (4 * VPR);
+  const int t = threadIdx.x;
+  const int c = t % VPR, g = (t / VPR) % 4, bi = t / (4 * VPR);
+  const size_t stride = (size_t)D.H * HD / 8;              // uint4 per token row
+  const uint4* base = reinterpret_cast<const uint4*>(frame) + (size_t)h * VPR + c;
+  for (int bb = b0; bb < b1; bb += BB) {
+    const int b = bb + bi;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    if (b < b1) {
+      const int ntok = block_len(D, b);
+      const int run = (ntok + 3) / 4;
+      const int t0 = g * run, t1 = min(ntok, t0 + run);
+      const uint4* src = base + (size_t)b * D.B * stride;
+      for (int k = t0; k < t1; k += 16) {
+        uint4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (k + u < t1) v[u] = __ldg(src + (size_t)(k + u) * stride);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          if (k + u < t1) {
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f2 = __bfloat1622float2(p2[i]);
+              acc[2 * i] += f2.x;
+              acc[2 * i + 1] += f2.y;
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[(bi * 4 + g) * HD + c * 8 + i] = acc[i];
+    __syncthreads();
+    for (int idx = t; idx < BB * HD; idx += kStreamThreads) {
+      const int bj = idx / HD, ch = idx % HD, bk = bb + bj;
+      if (bk < b1) {
+        const float* pp = part + bj * 4 * HD + ch;
+        const float sum = ((pp[0] + pp[HD]) + pp[2 * HD]) + pp[3 * HD];
+        const float inv = 1.0f / (float)block_len(D, bk);
+        out(bk, ch, sum * inv);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kStreamThreads, 2)
+select_stream_kernel(const __grid_constant__ StreamArgs a, const Dims D) {
+  extern __shared__ float4 sm4[];
+  float* smf = reinterpret_cast<float*>(sm4);
+  __shared__ int s_unit;
+  if (threadIdx.x == 0) s_unit = atomicAdd(&a.sync[0], 1);
+  __syncthreads();
+  const int unit = s_unit;
+  const int np = stream_parts(D), per = cdiv(D.nbpf, np);
+  const int UQ = D.H * D.Fc * np, UH = D.H * D.F * np;
+  int32_t* q_done = a.sync + 1;
+  int32_t* h_done = a.sync + 1 + D.H;
+  constexpr int VPR = HD / 8, BB = kStreamThreads / (4 * VPR);
+  float* part = smf;                                          // [BB][4][HD]
+  float* sk = part + BB * 4 * HD;                             // [kStreamBlocks][HD + 4]
+  float* sq = sk + kStreamBlocks * (HD + 4);                  // [nqb][HD + 4]
+
+  if (unit < UQ) {                                 // ---- pooled queries
+    const int h = unit / (D.Fc * np), r = unit % (D.Fc * np);
+    const int fc = r / np, p = r % np;
+    const int b0 = p * per, b1 = min(D.nbpf, b0 + per);
+    float* dst = a.q_blk + ((size_t)h * D.nqb + (size_t)fc * D.nbpf) * HD;
+    pool_part<HD>(a.q + (size_t)fc * D.T * D.H * HD, h, b0, b1, D, part,
+                  [&](int b, int ch, float v) { dst[(size_t)b * HD + ch] = v; });
+    cta_signal(&q_done[h]);
+  } else if (unit < UQ + UH) {                     // ---- pooled keys and their scores
+    const int u = unit - UQ;
+    const int h = u / (D.F * np), r = u % (D.F * np);
+    const int f = r / np, p = r % np;
+    const int b0 = p * per, b1 = min(D.nbpf, b0 + per);
+    pool_part<HD>(a.k_cache + (size_t)a.hist_slots[f] * D.T * D.H * HD, h, b0, b1, D, part,
+                  [&](int b, int ch, float v) { sk[(b - b0) * (HD + 4) + ch] = v; });
+    if (!cta_wait_count(&q_done[h], D.Fc * np, a.wait_limit_ns)) return;
+    const float4* qsrc = reinterpret_cast<const float4*>(a.q_blk + (size_t)h * D.nqb * HD);
+    for (int i = threadIdx.x; i < D.nqb * (HD / 4); i += kStreamThreads) {
+      const int qb = i / (HD / 4), c4 = i % (HD / 4);
+      reinterpret_cast<float4*>(sq + (size_t)qb * (HD + 4))[c4] = __ldcg(qsrc + i);
+    }
+    __syncthreads();
+    // thread task: one block x up to four query blocks (qg, qg + nqg, ...), each score one
+    // fma chain over the channels in order
+    const int nqg = cdiv(D.nqb, 4), nb = b1 - b0, NB = D.F * D.nbpf;
+    for (int task = threadIdx.x; task < nb * nqg; task += kStreamThreads) {
+      const int bl = task / nqg, qg = task % nqg;
+      const float4* kr = reinterpret_cast<const float4*>(sk + bl * (HD + 4));
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float4* qr[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int qb = min(qg + v * nqg, D.nqb - 1);
+        qr[v] = reinterpret_cast<const float4*>(sq + (size_t)qb * (HD + 4));
+      }
+#pragma unroll 8
+      for (int c4 = 0; c4 < HD / 4; ++c4) {
+        const float4 k = kr[c4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 q = qr[v][c4];
+          float x = acc[v];
+          x = fmaf(q.x, k.x, x); x = fmaf(q.y, k.y, x);
+          x = fmaf(q.z, k.z, x); x = fmaf(q.w, k.w, x);
+          acc[v] = x;
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int qb = qg + v * nqg;
+        if (qb < D.nqb) a.scores[((size_t)h * D.nqb + qb) * NB + (size_t)f * D.nbpf + b0 + bl] = acc[v];
+      }
+    }
+    cta_signal(&h_done[h]);
+  } else {                                         // ---- frame and block top-k, plans
+    const int u = unit - UQ - UH;
+    const int ng = cdiv(D.nqb, kFuseQb);
+    const int h = u / ng, g = u % ng;
+    if (!cta_wait_count(&h_done[h], D.F * np, a.wait_limit_ns)) return;
+    pick_group(a.scores, a.block_idx, a.plan, a.plan_cnt, D, h, g * kFuseQb, smf);
   }
 }
 

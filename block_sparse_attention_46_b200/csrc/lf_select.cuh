@@ -16,7 +16,8 @@ namespace lf {
 
 // ---------------------------------------------------------------------------------
 // (a) Pooling.  One CTA row (blockIdx.x) is one block of tokens: the first nqb rows are
-// the current chunk's query blocks, the next F*nbpf rows the history key blocks.  Each
+// the current chunk's query blocks, the next F*nbpf rows the history key blocks, and (when
+// the current chunk is sparse) the last nqb rows the current chunk's key blocks.  Each
 // thread owns 8 consecutive channels of the H*d-wide token row (one 16-byte load per
 // token), so a warp reads 512 contiguous bytes per token.  Sums are fp32 in a fixed
 // order: four consecutive runs of the block's tokens, each in token order, then the runs
@@ -29,6 +30,8 @@ struct PoolArgs {
   float* k_blk;                  // [H, F, nbpf, d]
   float* k_pool;                 // [n_slots, H, nbpf, d] pooled-key cache, or null: when
                                  // set, history blocks are written to their slot's rows
+  const __nv_bfloat16* k_cur;    // [ncur, H, d] current-chunk keys (with kc_blk)
+  float* kc_blk;                 // [H, nqb, d] current-chunk key block means, or null
   int hist_slots[LF_MAX_FRAMES];
 };
 
@@ -52,11 +55,14 @@ pool_blocks_kernel(const __grid_constant__ PoolArgs a, const Dims D) {
   int ntok;
   float* dst;
   const int h = (vec * 8) / D.d, c0 = (vec * 8) % D.d;
-  if (unit < D.nqb) {
-    const int f = unit / D.nbpf, b = unit % D.nbpf;
+  const int hist_end = D.nqb + D.F * D.nbpf;
+  if (unit < D.nqb || unit >= hist_end) {
+    const bool is_q = unit < D.nqb;                 // query block, or current key block
+    const int u = is_q ? unit : unit - hist_end;
+    const int f = u / D.nbpf, b = u % D.nbpf;
     ntok = block_len(D, b);
-    base = a.q + ((size_t)f * D.T + (size_t)b * D.B) * HD;
-    dst = a.q_blk + ((size_t)h * D.nqb + unit) * D.d + c0;
+    base = (is_q ? a.q : a.k_cur) + ((size_t)f * D.T + (size_t)b * D.B) * HD;
+    dst = (is_q ? a.q_blk : a.kc_blk) + ((size_t)h * D.nqb + u) * D.d + c0;
   } else {
     const int u = unit - D.nqb;
     const int f = u / D.nbpf, b = u % D.nbpf;
@@ -252,6 +258,48 @@ select_frames_kernel(const float* __restrict__ q_blk, const float* __restrict__ 
   }
   const uint32_t taken = warp_topk(sc, D.F, D.kf);
   warp_write_ascending(taken, D.F, frame_idx + ((size_t)h * D.nqb + qb) * D.kf, 0);
+}
+
+// ---------------------------------------------------------------------------------
+// Current-chunk block selection (sparse current chunk).  CTA = (group of 8 query blocks,
+// head); kc_blk[h] is staged in shared memory with a padded row pitch; warp w takes query
+// block qb = 8*blockIdx.x + w: lane c scores current blocks c, c+32, ... with a full-length
+// dot product in fixed order, the own block qb gets +inf so that it is always kept, and the
+// kc best are written ascending.
+// ---------------------------------------------------------------------------------
+template <int HD>
+__global__ void __launch_bounds__(kSelWarps * 32)
+select_current_kernel(const float* __restrict__ q_blk, const float* __restrict__ kc_blk,
+                      int32_t* __restrict__ cur_idx, const Dims D) {
+  extern __shared__ float4 sm4[];
+  float* sk = reinterpret_cast<float*>(sm4);
+  const int h = blockIdx.y;
+  const int pitch = D.d + 4;
+  float* sq = sk + (size_t)D.nqb * pitch;             // [kSelWarps][d]
+  for (int i = threadIdx.x; i < D.nqb * (D.d / 4); i += blockDim.x) {
+    const int c = i / (D.d / 4), c4 = i % (D.d / 4);
+    reinterpret_cast<float4*>(sk + (size_t)c * pitch)[c4] =
+        reinterpret_cast<const float4*>(kc_blk + ((size_t)h * D.nqb + c) * D.d)[c4];
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = blockIdx.x * kSelWarps + warp;
+  if (qb < D.nqb)
+    for (int c4 = lane; c4 < D.d / 4; c4 += 32)
+      reinterpret_cast<float4*>(sq + warp * D.d)[c4] =
+          reinterpret_cast<const float4*>(q_blk + ((size_t)h * D.nqb + qb) * D.d)[c4];
+  __syncthreads();
+  if (qb >= D.nqb) return;
+  float sc[kMaxPerLane];
+  const float* qv = sq + warp * D.d;
+#pragma unroll
+  for (int j = 0; j < kMaxPerLane; ++j) {
+    const int c = lane + 32 * j;
+    float s = -INFINITY;
+    if (c < D.nqb) s = c == qb ? INFINITY : dot_fixed<HD>(qv, sk + (size_t)c * pitch);
+    sc[j] = s;
+  }
+  const uint32_t taken = warp_topk(sc, D.nqb, D.kc);
+  warp_write_ascending(taken, D.nqb, cur_idx + ((size_t)h * D.nqb + qb) * D.kc, 0);
 }
 
 // ---------------------------------------------------------------------------------

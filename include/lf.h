@@ -29,8 +29,9 @@
  *    Pooled and score tensors are fp32, index tensors int32, all contiguous:
  *      q_blk  [H, n_qb, d]           k_blk [H, n_hist, n_bpf, d]    k_frm [H, n_hist, d]
  *      frame_idx [H, n_qb, kf]       block_idx [H, n_qb, kf*kb]      lse [H, n_cur_frames*T]
+ *      cur_idx [H, n_qb, kc]
  *    with T = tokens_per_frame, B = block, n_bpf = ceil(T/B), n_qb = n_cur_frames*n_bpf,
- *    kf = min(k_f, n_hist), kb = min(k_b, n_bpf).
+ *    kf = min(k_f, n_hist), kb = min(k_b, n_bpf), kc = min(k_c, n_qb).
  *  Blocks.  Block b of a frame covers tokens [b*B, min((b+1)*B, T)); the last block of a
  *    frame is shorter when B does not divide T.  Query block qb = frame*n_bpf + b.
  *    A global history block id is g = f*n_bpf + b, f being the history position.
@@ -59,7 +60,7 @@
 extern "C" {
 #endif
 
-#define LF_ABI_VERSION 1
+#define LF_ABI_VERSION 2
 
 /* status codes */
 #define LF_OK               0
@@ -75,7 +76,8 @@ extern "C" {
 #define LF_MAX_T            16384   /* tokens per frame                                 */
 #define LF_MAX_SELECTED     1024    /* kf * kb per query block                          */
 #define LF_MAX_PLAN         2048    /* key blocks per 128-row query tile:
-                                       n_sink * n_bpf + (block == 64 ? 2 : 1) * kf * kb  */
+                                       n_sink * n_bpf + (block == 64 ? 2 : 1) * (kc + kf*kb) */
+#define LF_MAX_CUR_BLOCKS   256     /* n_qb when the current chunk is sparse (k_c > 0)    */
 
 typedef struct lf_shape {
     int32_t H;                /* heads, >= 1                                              */
@@ -89,6 +91,8 @@ typedef struct lf_shape {
     int32_t k_f;              /* frames kept per query block (>= 1 when n_hist > 0)       */
     int32_t k_b;              /* blocks kept per chosen frame (>= 1 when n_hist > 0)      */
     float   scale;            /* softmax scale applied to q.k, normally 1/sqrt(d)         */
+    int32_t k_c;              /* current-chunk blocks kept per query block; 0 = the whole
+                                 current chunk (dense); kc = min(k_c, n_qb) otherwise      */
 } lf_shape;
 
 /* (a) Token compression [LF-gist 2.2 "token compression"; LF-yly 三, first stage].
@@ -167,25 +171,41 @@ int lf_select_chunk_cached(const lf_shape* shape, const void* q, const float* k_
                            const int32_t* hist_slots, int32_t* block_idx, void* workspace,
                            size_t workspace_bytes, cudaStream_t stream);
 
+/* Sparse current chunk [LF-yly 一: the first chunk, which has no history, tested at 80%
+ * sparsity, so the sparsity reaches the current chunk's own keys; LF-gist 2.2 token
+ * compression and inner-product block selection].  Requires shape->k_c >= 1 and
+ * n_qb <= LF_MAX_CUR_BLOCKS.  The current chunk's keys are mean-pooled per block exactly
+ * as the queries are (fp32, fixed order); query block qb keeps its own block qb and the
+ * kc - 1 other current blocks with the largest q_blk[h, qb] . kc_blk[h, c] (ties to the
+ * lower index).  cur_idx (device, [H, n_qb, kc]) receives the block ids c = frame*n_bpf
+ * + b, ascending.  workspace: at least lf_forward_workspace_size(shape) bytes, 256-byte
+ * aligned. */
+int lf_select_current(const lf_shape* shape, const void* q, const void* k_cur,
+                      int32_t* cur_idx, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
 /* Workspace bytes lf_block_sparse_attn needs for this shape (its per-tile key plans). */
 size_t lf_attn_workspace_size(const lf_shape* shape);
 
 /* (d) Block-sparse attention [LF-gist 2.2 "execution"; LF-yly 三, last stage].
  * For every query token of query block qb and head h, one joint softmax over
- *   - every key of the current chunk (k_cur, dense, no causal mask),
+ *   - the keys of the current chunk (k_cur): all of them (dense, no causal mask) when
+ *     shape->k_c == 0, else those of the current blocks listed in cur_idx[h, qb],
  *   - every key of every sink frame (k_cache at sink_slots) [RF],
  *   - the keys of the history blocks listed in block_idx[h, qb] (k_cache at hist_slots)
  * of scale * q.k, applied to the matching values.  out receives bf16; lse (nullable)
  * receives the natural-log normaliser log(sum exp(scale*q.k)) in fp32.
  * block_idx: [H, n_qb, kf*kb] ascending global ids (ignored, may be NULL, when
- * n_hist == 0).  Ids out of range or not ascending are recorded as LF_ERR_BAD_INDEX and
- * dropped.  Compute: tcgen05 bf16 MMAs with fp32 accumulation in tensor memory, fp32
- * online softmax. */
+ * n_hist == 0).  cur_idx: [H, n_qb, kc] ascending current block ids (ignored, may be
+ * NULL, when k_c == 0).  Ids out of range or not ascending are recorded as
+ * LF_ERR_BAD_INDEX and that list is dropped.  Compute: tcgen05 bf16 MMAs with fp32
+ * accumulation in tensor memory, fp32 online softmax. */
 int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur,
                          const void* v_cur, const void* k_cache, const void* v_cache,
                          const int32_t* hist_slots, const int32_t* sink_slots,
-                         const int32_t* block_idx, void* out, float* lse,
-                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                         const int32_t* block_idx, const int32_t* cur_idx, void* out,
+                         float* lse, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
 
 /* lf_block_sparse_attn for callers that cannot allocate device memory.
  *
@@ -208,6 +228,7 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
  *    on different streams, or from different host threads — race on it; serialise them.
  *  - A shape whose workspace (lf_attn_workspace_size) exceeds the array returns
  *    LF_ERR_WORKSPACE without launching anything.
+ *  - It takes no current-chunk list: a shape with k_c > 0 returns LF_ERR_INVALID_ARG.
  * Results are those of lf_block_sparse_attn. */
 size_t lf_noalloc_scratch_bytes(void);
 int lf_block_sparse_attn_noalloc(const lf_shape* shape, const void* q, const void* k_cur,
@@ -219,14 +240,16 @@ int lf_block_sparse_attn_noalloc(const lf_shape* shape, const void* q, const voi
 /* Workspace bytes lf_forward_chunk needs: pooled tensors, index lists and key plans. */
 size_t lf_forward_workspace_size(const lf_shape* shape);
 
-/* (a)->(b)->(c)->(d) in one call.  block_idx_out (nullable) receives the selected block
- * ids [H, n_qb, kf*kb]; lse is nullable.  With n_hist == 0 no selection runs and the
- * attention covers the current chunk and the sink frames. */
+/* (a)->(b)->(c)->(d) in one call (and, with k_c > 0, the current-chunk choice of
+ * lf_select_current).  block_idx_out (nullable) receives the selected block ids
+ * [H, n_qb, kf*kb], cur_idx_out (nullable) the kept current blocks [H, n_qb, kc]; lse is
+ * nullable.  With n_hist == 0 no history selection runs and the attention covers the
+ * current chunk and the sink frames. */
 int lf_forward_chunk(const lf_shape* shape, const void* q, const void* k_cur,
                      const void* v_cur, const void* k_cache, const void* v_cache,
                      const int32_t* hist_slots, const int32_t* sink_slots,
                      void* workspace, size_t workspace_bytes, void* out, float* lse,
-                     int32_t* block_idx_out, cudaStream_t stream);
+                     int32_t* block_idx_out, int32_t* cur_idx_out, cudaStream_t stream);
 
 /* Test hook, not part of the attention path (process-wide, not thread-safe; call it only
  * while no library work is queued).  Sets, for the attention launches that follow:

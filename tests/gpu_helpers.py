@@ -59,30 +59,53 @@ def gpu_select_blocks(ci, q_blk, k_blk, fidx):
     return bidx, bsc
 
 
-def gpu_attention(ci, t, block_idx):
+def gpu_select_current(ci, t):
+    sh = ci.shape
+    nbpf, nqb, kf, kb = lf.derived(sh)
+    cidx = torch.full((sh.H, nqb, lf.current_blocks(sh)), -7, dtype=torch.int32,
+                      device=t["q"].device)
+    lf.lf_select_current(sh, t["q"], t["k_cur"], cidx)
+    return cidx
+
+
+def gpu_attention(ci, t, block_idx, cur_idx=None):
     sh = ci.shape
     dev = t["q"].device
     out = torch.full_like(t["q"], float("nan"))
     lse = torch.full((sh.H, t["q"].shape[0]), float("nan"), device=dev)
-    bi = None
+    bi = ci_ = None
     if sh.n_hist > 0:
         bi = torch.as_tensor(np.asarray(block_idx), dtype=torch.int32).to(dev).contiguous()
+    if cur_idx is not None:
+        ci_ = torch.as_tensor(np.asarray(cur_idx), dtype=torch.int32).to(dev).contiguous()
     lf.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
-                            ci.hist_slots, ci.sink_slots, bi, out, lse)
+                            ci.hist_slots, ci.sink_slots, bi, out, lse, cur_idx=ci_)
     return out, lse
 
 
-def gpu_forward(ci, t):
+def gpu_forward(ci, t, with_cur=False):
+    """lf_forward_chunk; returns (out, lse, block_idx) or, with_cur, also cur_idx."""
     sh = ci.shape
     nbpf, nqb, kf, kb = lf.derived(sh)
     dev = t["q"].device
     out = torch.full_like(t["q"], float("nan"))
     lse = torch.full((sh.H, t["q"].shape[0]), float("nan"), device=dev)
     bidx = torch.full((sh.H, nqb, max(kf * kb, 1)), -7, dtype=torch.int32, device=dev)
+    kc = lf.current_blocks(sh)
+    cidx = torch.full((sh.H, nqb, max(kc, 1)), -7, dtype=torch.int32, device=dev)
     lf.lf_forward_chunk(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
                         ci.hist_slots, ci.sink_slots, out, lse,
-                        bidx if sh.n_hist > 0 else None)
+                        bidx if sh.n_hist > 0 else None, cur_idx_out=cidx if kc > 0 else None)
+    if with_cur:
+        return out, lse, bidx, cidx
     return out, lse, bidx
+
+
+def current_gaps(sc: np.ndarray, k_c: int) -> np.ndarray:
+    """Per (h, qb): the oracle's boundary gap of the current-chunk choice."""
+    H, nqb, _ = sc.shape
+    return np.array([[O.current_boundary_gap(list(sc[h, q]), q, min(k_c, nqb))
+                      for q in range(nqb)] for h in range(H)])
 
 
 def compare_indices(gpu_idx: np.ndarray, ora_idx: np.ndarray, gaps: np.ndarray):

@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(lib):
     raw = ctypes.CDLL(lf.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
-    assert lf.lf_abi_version() == 1
+    assert lf.lf_abi_version() == 2
 
 
 def _shape(**kw):
@@ -43,14 +43,15 @@ def _shape(**kw):
 FAKE = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
 
 
-def _attn(lib, shape, hist=(0, 1, 2, 3), sinks=(), ws=1 << 20, wsptr=FAKE, bidx=FAKE):
+def _attn(lib, shape, hist=(0, 1, 2, 3), sinks=(), ws=1 << 20, wsptr=FAKE, bidx=FAKE,
+          cidx=FAKE):
     sh = lf.make_shape(shape)
     h = (ctypes.c_int32 * max(len(hist), 1))(*hist)
     s = (ctypes.c_int32 * max(len(sinks), 1))(*sinks)
     return lib.lf_block_sparse_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE,
                                      ctypes.cast(h, ctypes.POINTER(ctypes.c_int32)),
-                                     ctypes.cast(s, ctypes.POINTER(ctypes.c_int32)), bidx, FAKE,
-                                     None, wsptr, ws, None)
+                                     ctypes.cast(s, ctypes.POINTER(ctypes.c_int32)), bidx, cidx,
+                                     FAKE, None, wsptr, ws, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -147,3 +148,23 @@ def test_debug_configure_validates_and_restores(lib):
     assert lib.lf_debug_configure(30_000_000_000, 0, 1) == 1          # above 20 s
     assert lib.lf_debug_configure(20_000_000, 0, 0) == 0
     assert lib.lf_debug_configure(0, 0, 1) == 0                       # defaults
+
+
+def test_sparse_current_chunk_validation(lib):
+    assert _attn(lib, _shape(k_c=-1)) == 1                             # negative k_c
+    assert _attn(lib, _shape(k_c=2), cidx=None) == 1                   # needs cur_idx
+    assert _attn(lib, _shape(k_c=2), ws=16) == 5                       # lists fine, ws small
+    # n_qb = 3 * ceil(16384 / 64) = 768 current blocks: above LF_MAX_CUR_BLOCKS
+    assert _attn(lib, _shape(T=16384, n_cur_frames=3, n_hist=0, n_slots=0, k_c=4),
+                 hist=()) == 2
+    # the fixed-scratch variant takes no current-chunk list
+    sh = lf.make_shape(_shape(k_c=2))
+    h = (ctypes.c_int32 * 4)(0, 1, 2, 3)
+    rc = lib.lf_block_sparse_attn_noalloc(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE,
+                                          ctypes.cast(h, ctypes.POINTER(ctypes.c_int32)), None,
+                                          FAKE, FAKE, None, None)
+    assert rc == 1
+    # lf_select_current needs k_c >= 1
+    rc = lib.lf_select_current(ctypes.byref(lf.make_shape(_shape())), FAKE, FAKE, FAKE, FAKE,
+                               1 << 20, None)
+    assert rc == 1

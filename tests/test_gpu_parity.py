@@ -223,3 +223,25 @@ def test_bad_block_index_is_reported_and_dropped(gpu_lib):
     torch.cuda.synchronize()
     assert gpu_lib.lf_device_status(True) == 6          # LF_ERR_BAD_INDEX
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("name", ["ragged_d64", "sinks_d128", "b128", "frames_1560_b64", "480p"])
+def test_forward_equals_stagewise_calls(gpu_lib, name):
+    """lf_forward_chunk (whose selection also writes the attention key plans) gives the
+    same bits as lf_select_chunk followed by lf_block_sparse_attn (whose plans are built
+    from the lists by plan_kernel): lists, plans and rounding agree."""
+    ci = W.p480(0) if name == "480p" else SMALL[name]()
+    sh = ci.shape
+    t = G.to_dev(ci)
+    nbpf, nqb, kf, kb = gpu_lib.derived(sh)
+    out, lse, bidx = G.gpu_forward(ci, t)
+    b2 = torch.full((sh.H, nqb, kf * kb), -7, dtype=torch.int32, device="cuda")
+    gpu_lib.lf_select_chunk(sh, t["q"], t["k_cache"], ci.hist_slots, b2)
+    out2 = torch.full_like(out, float("nan"))
+    lse2 = torch.full_like(lse, float("nan"))
+    gpu_lib.lf_block_sparse_attn(sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"], t["v_cache"],
+                                 ci.hist_slots, ci.sink_slots, b2, out2, lse2)
+    torch.cuda.synchronize()
+    assert torch.equal(bidx, b2)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+    assert gpu_lib.lf_device_status() == 0
