@@ -369,9 +369,10 @@ METRIC = "ms/chunk & effective TFLOP/s, hierarchical sparse attn, 480p chunk sha
 class ChunkRun:
     """Device tensors and C-ABI calls of one chunk of a workload."""
 
-    def __init__(self, lf, ci, dev):
+    def __init__(self, lf, ci, dev, e4m3=False):
         import torch
         self.lf, self.ci, self.sh = lf, ci, ci.shape
+        self.e4m3 = e4m3
         sh = self.sh
         nbpf, nqb, kf, kb = lf.derived(sh)
         self.t = {k: getattr(ci, k).to(dev) for k in ("q", "k_cur", "v_cur", "k_cache", "v_cache")}
@@ -384,6 +385,18 @@ class ChunkRun:
         self.lse = torch.empty(sh.H, self.t["q"].shape[0], device=dev)
         self.ws = torch.empty(max(lf.lf_attn_workspace_size(sh), 256), dtype=torch.uint8,
                               device=dev)
+        if e4m3:
+            # the cache's keys are quantised once (model state); the queries and the current
+            # chunk's keys every step, with the per-head key scales of the cache and chunk
+            t = self.t
+            self.q8 = torch.empty(t["q"].shape, dtype=torch.uint8, device=dev)
+            self.qs = torch.empty(t["q"].shape[0], sh.H, device=dev)
+            self.ks = torch.empty(sh.H, device=dev)
+            self.kc8 = torch.empty(t["k_cur"].shape, dtype=torch.uint8, device=dev)
+            self.kh8 = torch.empty(t["k_cache"].shape, dtype=torch.uint8, device=dev)
+            rows = t["k_cache"].view(-1, sh.H, sh.d)
+            lf.lf_e4m3_head_scales([t["k_cur"], rows], self.ks)
+            lf.lf_quantize_e4m3(rows, self.kh8.view(-1, sh.H, sh.d), head_scale=self.ks)
 
     def select(self):
         t = self.t
@@ -395,6 +408,14 @@ class ChunkRun:
 
     def attend(self):
         t = self.t
+        if self.e4m3:
+            self.lf.lf_quantize_e4m3(t["q"], self.q8, row_scale=self.qs)
+            self.lf.lf_quantize_e4m3(t["k_cur"], self.kc8, head_scale=self.ks)
+            self.lf.lf_block_sparse_attn_e4m3(
+                self.sh, self.q8, self.qs, self.kc8, t["v_cur"], self.kh8, t["v_cache"],
+                self.ks, self.ci.hist_slots, self.ci.sink_slots, self.bidx, self.out, self.lse,
+                self.ws, cur_idx=self.cidx if self.kc > 0 else None)
+            return
         self.lf.lf_block_sparse_attn(self.sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"],
                                      t["v_cache"], self.ci.hist_slots, self.ci.sink_slots,
                                      self.bidx, self.out, self.lse, self.ws,
@@ -408,7 +429,7 @@ class ChunkRun:
         # selection kernels (+ current-chunk pooling and choice) | plan, schedule, attn
         # (+ merge)
         return selection_launches(self.sh) + (2 if self.kc > 0 else 0) + 3 + \
-            (1 if tail_split(self.sh) else 0)
+            (1 if tail_split(self.sh) else 0) + (2 if self.e4m3 else 0)
 
 
 def capture(fn, stream, cap):
@@ -444,7 +465,10 @@ def run_lf(args, rank, world, local_rank):
         desc += f"; heads split over {world} ranks"
     else:
         chunks, desc = make_workload(args.config, rank)
-    runs = [ChunkRun(lf, ci, dev) for ci in chunks]
+    runs = [ChunkRun(lf, ci, dev, e4m3=args.e4m3) for ci in chunks]
+    if args.e4m3:
+        desc += "; stage (d) with e4m3 queries and keys (QK^T on the FP8 tensor cores, " \
+                "quantised in the step: queries per token, current keys per head) and bf16 values"
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     flush_sink = torch.empty((), dtype=torch.int64, device=dev)
 
@@ -521,7 +545,7 @@ def run_lf(args, rank, world, local_rank):
         job_flops = float(world * flops)
         value = weak_scaling_value(flops, world, ms_step)
 
-    single = len(runs) == 1 and runs[0].sh.n_hist > 0 and runs[0].kc == 0
+    single = len(runs) == 1 and runs[0].sh.n_hist > 0 and runs[0].kc == 0 and not args.e4m3
     inc = incremental_compression(lf, runs[0], args, stream, cap, ev, flush_l2, g_att) \
         if single else None
     abl = ablation_1d(lf, runs[0], args, stream, cap, ev, flush_l2) if single else None
@@ -536,7 +560,7 @@ def run_lf(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "strong" if args.shard == "heads" else "weak",
-        "vs_baseline": None, "dtype": "bf16",
+        "vs_baseline": None, "dtype": "e4m3 QK^T, bf16 PV" if args.e4m3 else "bf16",
         "data": "synthetic (seeded; per-frame key centroids, planted related frames)",
         "config": {"workload": desc, "chunks_per_step": n_chunks,
                    "l2": "flushed before every timed step (256 MB written, then read back)",
@@ -734,6 +758,8 @@ def main():
     ap.add_argument("--impl", default="lf", choices=["lf", "reference"])
     ap.add_argument("--config", default="480p", choices=CONFIG_NAMES)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e4m3", action="store_true",
+                    help="stage (d) with e4m3 queries and keys (lf_block_sparse_attn_e4m3)")
     ap.add_argument("--shard", default="chunks", choices=["chunks", "heads"],
                     help="chunks: one chunk per rank (weak scaling); heads: one chunk split "
                          "by heads over the ranks (strong scaling)")

@@ -22,6 +22,7 @@ __all__ = [
     "lf_noalloc_scratch_bytes", "lf_pooled_cache_bytes", "lf_pool_frames",
     "lf_select_chunk_cached", "lf_cag_schedule", "lf_select_chunk_1d",
     "lf_status_string", "lf_abi_version", "lf_debug_configure", "lf_select_current",
+    "lf_quantize_e4m3", "lf_e4m3_head_scales", "lf_block_sparse_attn_e4m3",
     "derived", "current_blocks", "LIB_PATH",
 ]
 
@@ -69,6 +70,13 @@ _SIGS = {
     "lf_abi_version": (ctypes.c_int, []),
     "lf_noalloc_scratch_bytes": (_SZ, []),
     "lf_debug_configure": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int, ctypes.c_int]),
+    "lf_block_sparse_attn_e4m3": (ctypes.c_int, [_SHP, _P, _P, _P, _P, _P, _P, _P, _I32P, _I32P,
+                                                 _P, _P, _P, _P, _P, _SZ, _P]),
+    "lf_quantize_e4m3": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P,
+                                        _P, _P, _P]),
+    "lf_e4m3_head_scales": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p),
+                                           ctypes.POINTER(ctypes.c_int64), ctypes.c_int32,
+                                           ctypes.c_int32, ctypes.c_int32, _P, _P]),
     "lf_pooled_cache_bytes": (_SZ, [_SHP]),
     "lf_cag_schedule": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                        ctypes.c_float, _I32P, ctypes.c_int32, ctypes.c_int32,
@@ -289,6 +297,43 @@ def lf_block_sparse_attn(shape, q, k_cur, v_cur, k_cache, v_cache, hist_slots, s
         ctypes.byref(sh), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_cache), _ptr(v_cache), hs, ss,
         _ptr(block_idx), _ptr(cur_idx), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)), "lf_block_sparse_attn")
+
+
+def lf_quantize_e4m3(x, x8, head_scale=None, row_scale=None, stream=None):
+    """e4m3 codes of x [rows, H, d] bf16 into x8 (uint8, same shape): per head with the given
+    scales [H], or per (row, head) with the scales written to row_scale [rows, H]."""
+    rows, H, d = x.shape
+    _check(load().lf_quantize_e4m3(_ptr(x), rows, H, d, _ptr(head_scale), _ptr(x8),
+                                   _ptr(row_scale), _stream(stream)), "lf_quantize_e4m3")
+
+
+def lf_e4m3_head_scales(xs, head_scale, stream=None):
+    """Per-head power-of-two scales over the bf16 tensors xs (each [rows, H, d])."""
+    n = len(xs)
+    H, d = xs[0].shape[-2], xs[0].shape[-1]
+    ptrs = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
+    rows = (ctypes.c_int64 * n)(*[x.numel() // (H * d) for x in xs])
+    for x in xs:
+        _ptr(x)
+    _check(load().lf_e4m3_head_scales(ptrs, rows, n, H, d, _ptr(head_scale), _stream(stream)),
+           "lf_e4m3_head_scales")
+
+
+def lf_block_sparse_attn_e4m3(shape, q8, q_scale, k_cur8, v_cur, k_cache8, v_cache, k_scale,
+                              hist_slots, sink_slots, block_idx, out, lse=None, workspace=None,
+                              stream=None, cur_idx=None):
+    """(d) with e4m3 queries and keys (QK^T on the FP8 tensor cores), bf16 values."""
+    sh = make_shape(shape)
+    hs, _k1 = _slots(hist_slots)
+    ss, _k2 = _slots(sink_slots)
+    if workspace is None:
+        workspace = torch.empty(max(lf_attn_workspace_size(shape), 256), dtype=torch.uint8,
+                                device=q8.device)
+    _check(load().lf_block_sparse_attn_e4m3(
+        ctypes.byref(sh), _ptr(q8), _ptr(q_scale), _ptr(k_cur8), _ptr(v_cur), _ptr(k_cache8),
+        _ptr(v_cache), _ptr(k_scale), hs, ss, _ptr(block_idx), _ptr(cur_idx), _ptr(out),
+        _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)),
+        "lf_block_sparse_attn_e4m3")
 
 
 def lf_noalloc_scratch_bytes() -> int:

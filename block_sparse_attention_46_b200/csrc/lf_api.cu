@@ -13,6 +13,7 @@
 #include "lf_select.cuh"
 #include "lf_attn.cuh"
 #include "lf_fused.cuh"
+#include "lf_fp8.cuh"
 
 using lf::Dims;
 
@@ -102,6 +103,33 @@ int encode_rows(CUtensorMap* m, const void* base, int HD, long long rows, int sl
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? LF_OK : LF_ERR_CUDA;
 }
+
+// e4m3 rows of H*d bytes: 2-D [rows, H*d] or 3-D [slots, T, H*d]; box = 128 bytes x 64 rows
+// (x 1 slot) -- one 128-byte swizzled row per token at d = 128; out-of-bounds bytes read as
+// zero.
+int encode_rows_e4m3(CUtensorMap* m, const void* base, int HD, long long rows, int slots) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return LF_ERR_CUDA;
+  const cuuint32_t rank = slots > 0 ? 3 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)rows, (cuuint64_t)(slots > 0 ? slots : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)HD, (cuuint64_t)HD * (cuuint64_t)rows};
+  cuuint32_t box[3] = {128, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LF_OK : LF_ERR_CUDA;
+}
+
+// e4m3 operands of the FP8 attention variant (null pointer: the bf16 path).
+struct F8Args {
+  const void* q8;          // [ncur, H, d] e4m3 codes
+  const float* q_scale;    // [ncur, H]
+  const void* k_cur8;      // [ncur, H, d]
+  const void* k_cache8;    // [n_slots, T, H, d]
+  const float* k_scale;    // [H]
+};
 
 // ---------------------------------------------------------------- launches
 // Pooling of the query blocks, the history key blocks (D.F frames) and, when kc_blk is
@@ -248,10 +276,10 @@ AttnWs carve_attn(const Dims& D, void* base, int n_sm) {
 
 size_t attn_ws_bytes(const Dims& D) { return carve_attn(D, nullptr, sm_count()).bytes; }
 
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8 = false>
 int launch_attn_t(const Dims& D, lf::AttnParams& p, int grid, cudaStream_t st) {
   using L = lf::AttnLayout<HD>;
-  auto kern = lf::attn_kernel<HD, BLK>;
+  auto kern = lf::attn_kernel<HD, BLK, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return LF_ERR_CUDA;
   // the in-kernel register split assumes the launch register count; never launch otherwise
@@ -266,7 +294,7 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
                 const void* k_cache, const void* v_cache, const int32_t* hist_slots,
                 const int32_t* sink_slots, const int32_t* block_idx, const int32_t* cur_idx,
                 void* out, float* lse, void* workspace, cudaStream_t st,
-                bool plans_ready = false) {
+                bool plans_ready = false, const F8Args* f8 = nullptr) {
   const int n_sm = sm_count();
   if (n_sm <= 0) return LF_ERR_CUDA;
   const AttnWs w = carve_attn(D, workspace, n_sm);
@@ -283,11 +311,22 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   lf::AttnParams p;
   memset(&p, 0, sizeof(p));
   const int HD = D.H * D.d;
-  if ((rc = encode_rows(&p.tm_q, q, HD, D.ncur, 0)) != LF_OK) return rc;
-  if ((rc = encode_rows(&p.tm_kc, k_cur, HD, D.ncur, 0)) != LF_OK) return rc;
+  if (f8 != nullptr) {                 // e4m3 queries and keys, bf16 values
+    if ((rc = encode_rows_e4m3(&p.tm_q, f8->q8, HD, D.ncur, 0)) != LF_OK) return rc;
+    if ((rc = encode_rows_e4m3(&p.tm_kc, f8->k_cur8, HD, D.ncur, 0)) != LF_OK) return rc;
+    p.q_scale = f8->q_scale;
+    p.k_scale = f8->k_scale;
+  } else {
+    if ((rc = encode_rows(&p.tm_q, q, HD, D.ncur, 0)) != LF_OK) return rc;
+    if ((rc = encode_rows(&p.tm_kc, k_cur, HD, D.ncur, 0)) != LF_OK) return rc;
+  }
   if ((rc = encode_rows(&p.tm_vc, v_cur, HD, D.ncur, 0)) != LF_OK) return rc;
   if (D.F + D.S > 0) {
-    if ((rc = encode_rows(&p.tm_kh, k_cache, HD, D.T, D.n_slots)) != LF_OK) return rc;
+    if (f8 != nullptr)
+      rc = encode_rows_e4m3(&p.tm_kh, f8->k_cache8, HD, D.T, D.n_slots);
+    else
+      rc = encode_rows(&p.tm_kh, k_cache, HD, D.T, D.n_slots);
+    if (rc != LF_OK) return rc;
     if ((rc = encode_rows(&p.tm_vh, v_cache, HD, D.T, D.n_slots)) != LF_OK) return rc;
   } else {   // no cache frames: the maps are never used; point them at the current chunk
     p.tm_kh = p.tm_kc;
@@ -308,7 +347,10 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   for (int i = 0; i < D.S; ++i) p.slots[i] = sink_slots[i];
   for (int i = 0; i < D.F; ++i) p.slots[D.S + i] = hist_slots[i];
   const int grid = sp.n_whole + sp.n_tail * sp.pieces;
-  if (D.d == 128)
+  if (f8 != nullptr)
+    rc = D.B == 64 ? launch_attn_t<128, 64, true>(D, p, grid, st)
+                   : launch_attn_t<128, 128, true>(D, p, grid, st);
+  else if (D.d == 128)
     rc = D.B == 64 ? launch_attn_t<128, 64>(D, p, grid, st) : launch_attn_t<128, 128>(D, p, grid, st);
   else
     rc = D.B == 64 ? launch_attn_t<64, 64>(D, p, grid, st) : launch_attn_t<64, 128>(D, p, grid, st);
@@ -665,6 +707,76 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
     return LF_ERR_WORKSPACE;
   return launch_attn(D, q, k_cur, v_cur, k_cache, v_cache, hist_slots, sink_slots, block_idx,
                      cur_idx, out, lse, workspace, stream);
+}
+
+int lf_block_sparse_attn_e4m3(const lf_shape* shape, const void* q8, const float* q_scale,
+                              const void* k_cur8, const void* v_cur, const void* k_cache8,
+                              const void* v_cache, const float* k_scale,
+                              const int32_t* hist_slots, const int32_t* sink_slots,
+                              const int32_t* block_idx, const int32_t* cur_idx, void* out,
+                              float* lse, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  Dims D;
+  int rc = make_dims(shape, &D);
+  if (rc != LF_OK) return rc;
+  if (D.d != 128) return LF_ERR_UNSUPPORTED;
+  if (q8 == nullptr || q_scale == nullptr || k_cur8 == nullptr || v_cur == nullptr ||
+      k_scale == nullptr || out == nullptr || !aligned(q8, 16) || !aligned(k_cur8, 16) ||
+      !aligned(v_cur, 16) || !aligned(out, 16) || !aligned(q_scale, 4) ||
+      !aligned(k_scale, 4) || (lse && !aligned(lse, 4)))
+    return LF_ERR_INVALID_ARG;
+  if (D.F + D.S > 0 && (k_cache8 == nullptr || v_cache == nullptr || !aligned(k_cache8, 16) ||
+                        !aligned(v_cache, 16)))
+    return LF_ERR_INVALID_ARG;
+  if (D.F > 0 && (block_idx == nullptr || !aligned(block_idx, 4))) return LF_ERR_INVALID_ARG;
+  if (D.kc > 0 && (cur_idx == nullptr || !aligned(cur_idx, 4))) return LF_ERR_INVALID_ARG;
+  if ((rc = check_slots(hist_slots, D.F, D.n_slots)) != LF_OK) return rc;
+  if ((rc = check_slots(sink_slots, D.S, D.n_slots)) != LF_OK) return rc;
+  const size_t need = attn_ws_bytes(D);
+  if (need == 0) return LF_ERR_CUDA;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need)
+    return LF_ERR_WORKSPACE;
+  const F8Args f8{q8, q_scale, k_cur8, k_cache8, k_scale};
+  return launch_attn(D, nullptr, nullptr, v_cur, nullptr, v_cache, hist_slots, sink_slots,
+                     block_idx, cur_idx, out, lse, workspace, stream, false, &f8);
+}
+
+int lf_quantize_e4m3(const void* x, int64_t rows, int32_t H, int32_t d, const float* head_scale,
+                     uint8_t* x8, float* row_scale, cudaStream_t stream) {
+  if (rows < 0 || H < 1 || (d != 64 && d != 128)) return LF_ERR_INVALID_ARG;
+  if (rows > ((int64_t)1 << 40) / ((int64_t)H * d)) return LF_ERR_UNSUPPORTED;
+  if (rows == 0) return LF_OK;
+  if (x == nullptr || x8 == nullptr || !aligned(x, 16) || !aligned(x8, 16) ||
+      (head_scale == nullptr && (row_scale == nullptr || !aligned(row_scale, 4))) ||
+      (head_scale != nullptr && !aligned(head_scale, 4)))
+    return LF_ERR_INVALID_ARG;
+  const long long units = rows * H;
+  const int warps = 8;
+  lf::quantize_e4m3_kernel<<<(unsigned)((units + warps - 1) / warps), warps * 32, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, H, d, head_scale, x8, row_scale);
+  return cuda_status(cudaGetLastError());
+}
+
+int lf_e4m3_head_scales(const void* const* xs, const int64_t* rows, int32_t n, int32_t H,
+                        int32_t d, float* head_scale, cudaStream_t stream) {
+  if (n < 1 || n > 16 || xs == nullptr || rows == nullptr || H < 1 || (d != 64 && d != 128) ||
+      head_scale == nullptr || !aligned(head_scale, 4))
+    return LF_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (rows[i] < 0 || (rows[i] > 0 && (xs[i] == nullptr || !aligned(xs[i], 16))))
+      return LF_ERR_INVALID_ARG;
+  // head_scale first holds the amax bit patterns, then (in place) the scales
+  if (cudaMemsetAsync(head_scale, 0, (size_t)H * sizeof(float), stream) != cudaSuccess)
+    return LF_ERR_CUDA;
+  unsigned int* bits = reinterpret_cast<unsigned int*>(head_scale);
+  for (int i = 0; i < n; ++i) {
+    if (rows[i] == 0) continue;
+    const long long blocks = std::min<long long>((rows[i] + 255) / 256, 1024);
+    lf::head_amax_kernel<<<dim3((unsigned)blocks, H), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(xs[i]), rows[i], H, d, bits);
+  }
+  lf::head_scale_kernel<<<(H + 127) / 128, 128, 0, stream>>>(bits, H, head_scale);
+  return cuda_status(cudaGetLastError());
 }
 
 size_t lf_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }

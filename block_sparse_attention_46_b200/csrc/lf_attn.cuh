@@ -290,6 +290,8 @@ struct AttnParams {
   int pieces;
   float* part_o;       // [n_tail * pieces, 128, d] unnormalised O
   float* part_ml;      // [n_tail * pieces, 2, 128] row max (log2 units) and row sum
+  const float* q_scale;       // e4m3 variant: [ncur, H] query scales (tm_q and tm_kc/tm_kh
+  const float* k_scale;       // then map e4m3 Q and K), [H] key scales; else unused
   uint64_t wait_limit_ns;     // limit of every bounded wait of the launch (kWaitLimitNs)
   int debug_stall;     // test hook: when set, CTA 0 never arms its Q barrier, so its
                        // first wait runs out (the timeout and drain path)
@@ -334,15 +336,35 @@ __device__ __forceinline__ int ring_tile(int q, bool& isK) {
   return (q + 1) >> 1;
 }
 
+// Maximum of N (64 or 128) values: eight independent chains of three-input max.
+template <int N>
+__device__ __forceinline__ float row_max(const float* v) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = fmax3f(v[k], v[8 + k], v[16 + k]);
+#pragma unroll
+  for (int i = 24; i < N - 8; i += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = fmax3f(m[k], v[i + k], v[i + 8 + k]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = fmaxf(m[k], v[N - 8 + k]);
+  return fmaxf(fmax3f(m[0], m[1], m[2]), fmax3f(fmax3f(m[3], m[4], m[5]), m[6], m[7]));
+}
+
 constexpr int kSoftmaxWarps = 8;          // two warpgroups, alternate key tiles
 // Register split: launched at 168 per thread (384 threads); the load/MMA warpgroup gives
 // registers to the two softmax warpgroups: 128 x 72 + 256 x 216 <= 384 x 168.
 constexpr int kLaunchRegs = 168, kLowRegs = 72, kHighRegs = 216;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kAttnThreads * kLaunchRegs, "register split");
 
-template <int HD, int BLK>
+// F8: queries and keys are e4m3 codes (one byte per element, 128-byte rows at d = 128, one
+// swizzled region per 128-row tile), S = Q K^T by tcgen05.mma kind::f8f6f4 (exact products,
+// fp32 accumulation) and the scales enter the softmax's per-row factor; V, P and the PV
+// MMAs are as in the bf16 path.
+template <int HD, int BLK, bool F8 = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
+  static_assert(!F8 || HD == 128, "the e4m3 path has d = 128");
   using L = AttnLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -421,7 +443,12 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   if (warp == 0 && lane == 0) {
     uint64_t* full = &bars[kBarRing];
     uint64_t* empty = &bars[kBarRing + L::kSlots];
-    if (!(P.debug_stall && blockIdx.x == 0)) {
+    if (F8 && !(P.debug_stall && blockIdx.x == 0)) {
+      mbar_arrive_expect_tx(&bars[kBarQ], 128 * HD);         // e4m3: one byte per element
+      uint8_t* dst = smem + L::kQ;
+      tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD, tokA);
+      tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD, BLK == 64 ? tokB : tokA + 64);
+    } else if (!(P.debug_stall && blockIdx.x == 0)) {
       mbar_arrive_expect_tx(&bars[kBarQ], L::kQBytes);
       for (int c = 0; c < L::NH; ++c) {
         uint8_t* dst = smem + L::kQ + c * L::kRegion;
@@ -441,16 +468,19 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort, P.wait_limit_ns)) break;
       const int j = j0 + l;
       LF_TR(isK ? 0 : 1, l);
-      mbar_arrive_expect_tx(&full[slot], L::kStageBytes);
+      const bool f8 = F8 && isK;                     // an e4m3 key tile: one 16 KB region
+      const int nreg = f8 ? 1 : L::NH;
+      const int xcol = f8 ? h * HD : 0;               // x coordinate base: bytes / elements
+      mbar_arrive_expect_tx(&full[slot], f8 ? 128 * HD : L::kStageBytes);
       uint8_t* st = smem + L::kRing + slot * L::kStageBytes;
       const CUtensorMap* tm_cur = isK ? &P.tm_kc : &P.tm_vc;
       const CUtensorMap* tm_hist = isK ? &P.tm_kh : &P.tm_vh;
       for (int box = 0; box < 2; ++box) {
         if (j < n_dense) {
           const int row = j * 128 + box * 64;
-          for (int c = 0; c < L::NH; ++c)
+          for (int c = 0; c < nreg; ++c)
             tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
-                        h * HD + c * 64, row);
+                        f8 ? xcol : h * HD + c * 64, row);
         } else {
           const int u = j - n_dense;
           int slot_id = 0, tok = 0;
@@ -466,13 +496,13 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
             // a block of the current chunk (2-D map), or padding: rows from ncur on are
             // out of bounds and read as zero (the columns are masked anyway)
             const int row = p < 0 ? D.ncur : (p - D.S - D.F) * D.T + tok;
-            for (int c = 0; c < L::NH; ++c)
+            for (int c = 0; c < nreg; ++c)
               tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
-                          h * HD + c * 64, row);
+                          f8 ? xcol : h * HD + c * 64, row);
           } else {
-            for (int c = 0; c < L::NH; ++c)
+            for (int c = 0; c < nreg; ++c)
               tma_load_3d(st + c * L::kRegion + box * 64 * 128, tm_hist, &full[slot],
-                          h * HD + c * 64, tok, slot_id);
+                          f8 ? xcol : h * HD + c * 64, tok, slot_id);
           }
         }
       }
@@ -490,7 +520,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   // P_l was read from.  tcgen05.mma runs in issue order, so S_{l+2} overwrites P_l only
   // after PV_l has consumed it, and the completion of S_{l+2} implies that of PV_l.
   else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, 0, 1);
     const uint32_t q_base = smem_u32(smem + L::kQ);
     const uint32_t ring_base = smem_u32(smem + L::kRing);
@@ -505,11 +535,18 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       tc_fence_after();
       const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
       const uint32_t k_addr = ring_base + slot * L::kStageBytes;
+      if constexpr (F8) {
 #pragma unroll
-      for (int ks = 0; ks < HD / 16; ++ks) {
-        const uint32_t off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
-        mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
-                    smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < HD / 32; ++ks)          // 32 e4m3 elements = 32 bytes per MMA
+          mma_e4m3_ss(d_tmem, smem_desc_sw128(q_base + ks * 32, 16, 1024),
+                      smem_desc_sw128(k_addr + ks * 32, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
+          mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
+                      smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+        }
       }
       mma_commit(&bars[kBarSFull + s]);
       mma_commit(&empty[slot]);
@@ -558,7 +595,14 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     const uint32_t row_bit = (BLK == 64 && r >= 64) ? 2u : 1u;
     const uint32_t s_col = wg ? L::kColS1 : L::kColS0;
     const uint32_t o_col = wg ? L::kColO1 : L::kColO0;
-    const float c = D.scale * 1.4426950408889634f;         // scale * log2(e)
+    // scale * log2(e), times the row's query scale and the head's key scale for e4m3 Q/K
+    float c = D.scale * 1.4426950408889634f;
+    if constexpr (F8) {
+      const int qb = BLK == 64 ? (r < 64 ? qbA : qbB) : qbA, i = BLK == 64 ? (r & 63) : r;
+      const bool valid = qb >= 0 && i < block_len(D, qb % D.nbpf);
+      const int tok = valid ? (qb / D.nbpf) * D.T + (qb % D.nbpf) * BLK + i : 0;
+      c *= (valid ? P.q_scale[(size_t)tok * D.H + h] : 1.0f) * P.k_scale[h];
+    }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int n_mine = 0;                                        // PVs into this group's O
@@ -601,24 +645,30 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
           v1 = max(0, len - 64);
         }
       }
-      if (v0 < 64 || v1 < 64) {
+      // row maximum over the valid columns (v0, v1 are warp-uniform: a warp's 32 rows
+      // belong to one query block).  A half that is wholly valid or wholly masked needs no
+      // per-column masking (a wholly masked half is left out of the maximum and skips its
+      // exponentials below); only a partly valid half (a short last block of a frame, or
+      // the end of the current chunk) is masked column by column.
+      float m_raw;
+      const bool full0 = v0 == 64, full1 = v1 == 64;
+      if ((v0 != 0 && !full0) || (v1 != 0 && !full1)) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           if (i >= v0) sv[i] = -INFINITY;
           if (i >= v1) sv[64 + i] = -INFINITY;
         }
+        m_raw = row_max<128>(sv);
+      } else if (full0 && full1) {
+        m_raw = row_max<128>(sv);
+      } else if (full0) {
+        m_raw = row_max<64>(sv);
+      } else if (full1) {
+        m_raw = row_max<64>(sv + 64);
+      } else {
+        m_raw = -INFINITY;
       }
-      float mx8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(sv[k], sv[8 + k], sv[16 + k]);
-#pragma unroll
-      for (int i = 24; i < 120; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(mx8[k], sv[i + k], sv[i + 8 + k]);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], sv[120 + k]);
-      const float m_tile = fmaxf(fmax3f(mx8[0], mx8[1], mx8[2]),
-                                 fmax3f(fmax3f(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * c;
+      const float m_tile = m_raw * c;
       float m_new = m_run;
       bool resc = false;
       if (m_tile > m_run + 8.0f) { m_new = m_tile; resc = true; }

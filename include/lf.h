@@ -207,6 +207,40 @@ int lf_block_sparse_attn(const lf_shape* shape, const void* q, const void* k_cur
                          float* lse, void* workspace, size_t workspace_bytes,
                          cudaStream_t stream);
 
+/* FP8 (e4m3) variant of (d) [LF-yly 五 deploys the video model with FP8, activations
+ * quantised per token; using e4m3 for the attention's QK^T operands is this library's
+ * extension].  The same attention as lf_block_sparse_attn (d = 128 only) on dequantised
+ * queries and keys: q8 [n_cur_frames*T, H, d] and k_cur8 / k_cache8 (k_cur / k_cache
+ * layouts) are e4m3 codes as written by lf_quantize_e4m3; q_scale [n_cur_frames*T, H]
+ * holds one power-of-two scale per (token, head), k_scale [H] one per head for every key
+ * the call can attend to; v_cur and v_cache stay bf16.  S = Q K^T runs on tcgen05.mma
+ * kind::f8f6f4 (exact products, fp32 accumulation); the scales enter the softmax's
+ * per-row factor, so the result is that of the dequantised operands within the bf16
+ * path's rounding.  Workspace: lf_attn_workspace_size.  LF_ERR_UNSUPPORTED for d != 128. */
+int lf_block_sparse_attn_e4m3(const lf_shape* shape, const void* q8, const float* q_scale,
+                              const void* k_cur8, const void* v_cur, const void* k_cache8,
+                              const void* v_cache, const float* k_scale,
+                              const int32_t* hist_slots, const int32_t* sink_slots,
+                              const int32_t* block_idx, const int32_t* cur_idx, void* out,
+                              float* lse, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/* e4m3 quantisation of a bf16 tensor x [rows, H, d] (d in {64, 128}) into x8 (same layout,
+ * one byte per element): each value is divided by its group's scale (a power of two, so
+ * exactly) and rounded to the nearest e4m3 value, ties to the even code.  head_scale
+ * non-null: the groups are the heads, with the given scales [H] (powers of two large
+ * enough that |x| / scale <= 448; larger values saturate to 448); else the groups are the
+ * (row, head) pairs and their scales -- the smallest 2^e with max|x| <= 448 * 2^e, 1 for an
+ * all-zero row -- are written to row_scale [rows, H]. */
+int lf_quantize_e4m3(const void* x, int64_t rows, int32_t H, int32_t d, const float* head_scale,
+                     uint8_t* x8, float* row_scale, cudaStream_t stream);
+
+/* Per-head power-of-two scales over n (1..16) bf16 tensors xs[i] [rows[i], H, d] (HOST
+ * arrays of device pointers and row counts): head_scale[h] (device, [H]) = the smallest
+ * 2^e with max |x[., h, .]| <= 448 * 2^e over all of them (1 when all are zero). */
+int lf_e4m3_head_scales(const void* const* xs, const int64_t* rows, int32_t n, int32_t H,
+                        int32_t d, float* head_scale, cudaStream_t stream);
+
 /* lf_block_sparse_attn for callers that cannot allocate device memory.
  *
  * No counterpart in the paper: this is a packaging variant of (d).  Some callers cannot

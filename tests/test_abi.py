@@ -168,3 +168,20 @@ def test_sparse_current_chunk_validation(lib):
     rc = lib.lf_select_current(ctypes.byref(lf.make_shape(_shape())), FAKE, FAKE, FAKE, FAKE,
                                1 << 20, None)
     assert rc == 1
+
+
+def test_e4m3_entry_points_validate(lib):
+    sh = lf.make_shape(_shape(d=64))
+    h = (ctypes.c_int32 * 4)(0, 1, 2, 3)
+    hp = ctypes.cast(h, ctypes.POINTER(ctypes.c_int32))
+    rc = lib.lf_block_sparse_attn_e4m3(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                       hp, None, FAKE, None, FAKE, None, FAKE, 1 << 20, None)
+    assert rc == 2                                                    # d = 64: unsupported
+    sh = lf.make_shape(_shape(d=128))
+    rc = lib.lf_block_sparse_attn_e4m3(ctypes.byref(sh), FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                       hp, None, FAKE, None, FAKE, None, FAKE, 1 << 20, None)
+    assert rc == 1                                                    # no query scales
+    assert lib.lf_quantize_e4m3(FAKE, 10, 2, 96, None, FAKE, FAKE, None) == 1     # d = 96
+    assert lib.lf_quantize_e4m3(FAKE, 10, 2, 64, None, FAKE, None, None) == 1     # no row_scale
+    assert lib.lf_quantize_e4m3(FAKE, 0, 2, 64, None, FAKE, FAKE, None) == 0      # nothing to do
+    assert lib.lf_e4m3_head_scales(None, None, 0, 2, 64, FAKE, None) == 1
