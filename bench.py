@@ -86,22 +86,15 @@ def tail_split(shape, n_sm=148) -> bool:
 
 
 def selection_launches(shape) -> int:
-    """Kernels one lf_select_chunk call launches (mirrors the library's rule): one when the
-    single-launch selection applies, else pooling, block scores and pick when the fused
-    path applies, else pooling, frame pooling, frame selection and block selection."""
+    """Kernels one lf_select_chunk call launches (mirrors the library's rule): pooling,
+    block scores and pick when the fused path applies, else pooling, frame pooling, frame
+    selection and block selection."""
     if shape.n_hist <= 0:
         return 0
     nbpf = -(-shape.T // shape.block)
-    nqb = shape.n_cur_frames * nbpf
     kf, kb = min(shape.k_f, shape.n_hist), min(shape.k_b, nbpf)
     fused = (shape.n_hist * nbpf <= 2048 and kf * kb <= 256 and shape.n_hist <= 256
              and nbpf <= 256)
-    pick_smem = 2 * shape.n_hist * nbpf * 4 + 2 * kf * kb * 4 + 2 * kf * 4
-    bb = 256 // (4 * (shape.d // 8))
-    stream_smem = max(bb * 4 * shape.d * 4 + 16 * (shape.d + 4) * 4 + nqb * (shape.d + 4) * 4,
-                      pick_smem)
-    if fused and getattr(shape, "k_c", 0) == 0 and stream_smem <= 227 * 1024:
-        return 1
     return 3 if fused else 4
 
 
@@ -585,8 +578,7 @@ def run_lf(args, rank, world, local_rank):
         line["roofline_selection"] = {
             "bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": sel_gbs / pk["hbm_gbs"],
-            "kernels": "lf_select_chunk: select_stream_kernel (pooling, scores and picks in one "
-                       "launch) where the shape allows it",
+            "kernels": "pool_blocks + block_scores + select_pick (lf_select_chunk)",
             "peak_source": f"{src} hbm_gbs"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, dt, cores, n = oracle_sample(chunks, budget_s=10.0)

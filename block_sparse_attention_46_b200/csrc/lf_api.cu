@@ -362,7 +362,7 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
 // forward workspace carve-up
 struct FwdWs {
   float *q_blk, *k_blk, *k_frm, *scores, *kc_blk;
-  int32_t *frame_idx, *block_idx, *cur_idx, *sync;
+  int32_t *frame_idx, *block_idx, *cur_idx;
   void* attn;
   size_t bytes;
 };
@@ -380,7 +380,6 @@ FwdWs carve(const Dims& D, void* base) {
   w.block_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.nsel * 4));
   w.kc_blk = reinterpret_cast<float*>(take((size_t)D.H * (D.kc > 0 ? D.nqb : 0) * D.d * 4));
   w.cur_idx = reinterpret_cast<int32_t*>(take((size_t)D.H * D.nqb * D.kc * 4));
-  w.sync = reinterpret_cast<int32_t*>(take((size_t)(1 + 2 * D.H) * 4));
   w.attn = take(attn_ws_bytes(D));
   w.bytes = off;
   return w;
@@ -423,60 +422,15 @@ int launch_scores_pick(const Dims& D, const FwdWs& w, const float* k_pool,
   return cuda_status(cudaGetLastError());
 }
 
-// Whether stages (a)-(c) run as the single-launch selection kernel.
-bool stream_ok(const Dims& D) {
-  if (D.kc > 0 || !lf::fused_select_ok(D)) return false;
-  const size_t smem = D.d == 128 ? lf::stream_smem<128>(D) : lf::stream_smem<64>(D);
-  return smem <= kMaxSmem;
-}
-
-// Stages (a)-(c) in one launch (lf::select_stream_kernel): the work counters are zeroed,
-// then every pooling, scoring and pick unit runs in ticket order.
-int launch_stream(const Dims& D, const void* q, const void* k_cache, const int32_t* hist_slots,
-                  const FwdWs& w, const AttnWs& aw, int32_t* bidx, cudaStream_t stream) {
-  if (cudaMemsetAsync(w.sync, 0, (size_t)(1 + 2 * D.H) * sizeof(int32_t), stream) != cudaSuccess)
-    return LF_ERR_CUDA;
-  lf::StreamArgs a{};
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
-  a.q_blk = w.q_blk;
-  a.scores = w.scores;
-  a.block_idx = bidx;
-  a.plan = aw.plan;
-  a.plan_cnt = aw.plan_cnt;
-  a.sync = w.sync;
-  a.wait_limit_ns = g_dbg_wait_limit_ns;
-  for (int f = 0; f < D.F; ++f) a.hist_slots[f] = hist_slots[f];
-  const int np = lf::stream_parts(D);
-  const int units = D.H * (D.Fc + D.F) * np + D.H * lf::cdiv(D.nqb, lf::kFuseQb);
-  auto kern = D.d == 128 ? lf::select_stream_kernel<128> : lf::select_stream_kernel<64>;
-  const size_t smem = D.d == 128 ? lf::stream_smem<128>(D) : lf::stream_smem<64>(D);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return LF_ERR_CUDA;
-  kern<<<units, lf::kStreamThreads, smem, stream>>>(a, D);
-  return cuda_status(cudaGetLastError());
-}
-
-// Stages (a)-(c) into `bidx`: the single-launch selection when the shape allows it, else
-// pooling and the pick kernel, else the separate frame-pooling, frame-selection and
-// block-selection kernels.  The first two also write the attention key plans into the
-// workspace (*plans_ready).
+// Stages (a)-(c) into `bidx`: pooling, then the fused selection (which also writes the
+// attention key plans into the workspace, *plans_ready) when the shape allows it, else the
+// separate frame-pooling, frame-selection and block-selection kernels.
 int run_select(const Dims& D, const void* q, const void* k_cache, const int32_t* hist_slots,
                const FwdWs& w, int32_t* bidx, cudaStream_t stream, bool* plans_ready,
                const void* k_cur = nullptr) {
   int rc;
   *plans_ready = false;
   float* kc_blk = k_cur != nullptr ? w.kc_blk : nullptr;   // also pool the current keys
-  if (k_cur == nullptr && stream_ok(D)) {
-    const int n_sm = sm_count();
-    if (n_sm <= 0) return LF_ERR_CUDA;
-    if ((rc = launch_stream(D, q, k_cache, hist_slots, w, carve_attn(D, w.attn, n_sm), bidx,
-                            stream)) != LF_OK)
-      return rc;
-    *plans_ready = true;
-    return LF_OK;
-  }
   if (lf::fused_select_ok(D) && lf::fused_select_smem(D) <= kMaxSmem) {
     if ((rc = launch_compress(D, q, k_cache, hist_slots, w.q_blk, w.k_blk, nullptr, stream,
                               k_cur, kc_blk)) != LF_OK)

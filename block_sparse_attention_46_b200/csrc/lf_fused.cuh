@@ -156,7 +156,16 @@ __device__ __forceinline__ void pick_group(const float* __restrict__ scores,
     // the group's rows of the score matrix are contiguous: [qb0, qb0 + kFuseQb) x NB
     const int ng = min(kFuseQb, D.nqb - qb0);
     const float* src = scores + ((size_t)h * D.nqb + qb0) * NB;
-    for (int i = threadIdx.x; i < ng * NB; i += blockDim.x) sc[i] = __ldcg(src + i);
+    const int n = ng * NB, tid = threadIdx.x, nt = blockDim.x;
+    int i = tid;
+    for (; i + 7 * nt < n; i += 8 * nt) {          // eight L2 loads in flight per thread
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + i + u * nt);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sc[i + u * nt] = v[u];
+    }
+    for (; i < n; i += nt) sc[i] = __ldcg(src + i);
   }
   __syncthreads();
 
@@ -267,226 +276,6 @@ select_pick_kernel(const float* __restrict__ scores, int32_t* __restrict__ block
   extern __shared__ float4 sm4[];
   pick_group(scores, block_idx, plan, plan_cnt, D, blockIdx.y, blockIdx.x * kFuseQb,
              reinterpret_cast<float*>(sm4));
-}
-
-// ---------------------------------------------------------------------------------
-// Stages (a)-(c) in one launch.  Work units are handed out in order by an atomic ticket:
-//   [0, UQ)            pooling of the query blocks of (head, current frame, part),
-//   [UQ, UQ + UH)      pooling of the key blocks of (head, history frame, part) and their
-//                      scores against every pooled query block of the head,
-//   [UQ + UH, total)   the pick of (head, group of kFuseQb query blocks).
-// A part is a run of at most kStreamBlocks consecutive blocks of one frame, one head's d
-// channels.  A history unit waits until its head's query units are done, a pick unit until
-// its head's history units are done; the units waited for hold lower tickets, so they were
-// taken by CTAs that already run, and every wait ends (each is also bounded in time).
-// Sums are in the order of pool_blocks_kernel (four runs of a block's tokens, each in token
-// order, then the runs in order, times the reciprocal of the length) and of
-// block_scores_kernel (one fma chain over the channels in order), so pooled values, scores,
-// lists and plans are bit-identical to the three-kernel path.
-// ---------------------------------------------------------------------------------
-constexpr int kStreamThreads = 256;
-constexpr int kStreamBlocks = 16;          // blocks per pooling part, at most
-
-struct StreamArgs {
-  const __nv_bfloat16* q;        // [ncur, H, d]
-  const __nv_bfloat16* k_cache;  // [n_slots, T, H, d]
-  float* q_blk;                  // [H, nqb, d]
-  float* scores;                 // [H, nqb, F * nbpf]
-  int32_t* block_idx;            // [H, nqb, nsel]
-  uint32_t* plan;                // key plans, or null (lists only)
-  int32_t* plan_cnt;
-  int32_t* sync;                 // [1 + 2H], zero at launch: ticket, q_done[H], hist_done[H]
-  uint64_t wait_limit_ns;
-  int hist_slots[LF_MAX_FRAMES];
-};
-
-__host__ __device__ inline int stream_parts(const Dims& D) { return cdiv(D.nbpf, kStreamBlocks); }
-
-template <int HD>
-__host__ __device__ inline size_t stream_smem(const Dims& D) {
-  const size_t pool = (size_t)kStreamBlocks * (HD + 4) * 4 + (size_t)D.nqb * HD * 4;
-  const size_t pick = fused_select_smem(D);
-  return pool > pick ? pool : pick;
-}
-
-// Waits (thread 0, then the whole CTA) until *counter reaches target; false on timeout.
-__device__ __forceinline__ bool cta_wait_count(const int32_t* counter, int target,
-                                               uint64_t limit_ns) {
-  __shared__ int s_ok;
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    if (*reinterpret_cast<const volatile int32_t*>(counter) < target) {
-      const uint64_t t0 = globaltimer_ns();
-      while (*reinterpret_cast<const volatile int32_t*>(counter) < target) {
-        if (globaltimer_ns() - t0 > limit_ns) {
-          record_status(LF_ERR_TIMEOUT);
-          ok = 0;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __threadfence();
-    s_ok = ok;
-  }
-  __syncthreads();
-  return s_ok != 0;
-}
-
-// Publishes this CTA's global writes, then adds one to *counter.
-__device__ __forceinline__ void cta_signal(int32_t* counter) {
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) atomicAdd(counter, 1);
-}
-
-// Pools blocks [b0, b1) of one frame for head h (frame = token 0 of the frame, row pitch
-// H*d bf16) and hands each block mean to out(b, channel, value).  A warp task is one block
-// and 8 of the head's 16-byte channel groups: lane = 4 * group + run, so the four runs of
-// a block's tokens (each summed in token order) sit in four adjacent lanes and are added
-// in run order with shuffles; no shared memory and no CTA barrier between tasks.
-template <int HD, typename Out>
-__device__ __forceinline__ void pool_part(const __nv_bfloat16* __restrict__ frame, int h,
-                                          int b0, int b1, const Dims& D, Out out) {
-  constexpr int VPR = HD / 8;                              // 16-byte groups per head row
-  constexpr int HALVES = VPR / 8;                          // warp tasks per block
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane & 3, cl = lane >> 2;
-  const size_t stride = (size_t)D.H * HD / 8;              // uint4 per token row
-  const int ntask = (b1 - b0) * HALVES;
-  for (int task = warp; task < ntask; task += kStreamThreads / 32) {
-    const int b = b0 + task / HALVES, c = (task % HALVES) * 8 + cl;
-    const int ntok = block_len(D, b);
-    const int run = (ntok + 3) / 4;
-    const int t0 = g * run, t1 = min(ntok, t0 + run);
-    const uint4* src = reinterpret_cast<const uint4*>(frame) + (size_t)h * VPR + c +
-                       (size_t)b * D.B * stride;
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int k = t0; k < t1; k += 8) {
-      uint4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (k + u < t1) v[u] = __ldg(src + (size_t)(k + u) * stride);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (k + u < t1) {
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f2 = __bfloat1622float2(p2[i]);
-            acc[2 * i] += f2.x;
-            acc[2 * i + 1] += f2.y;
-          }
-        }
-      }
-    }
-    // ((run0 + run1) + run2) + run3, in lane g = 0 of each group of four lanes
-    const float inv = 1.0f / (float)ntok;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float r1 = __shfl_down_sync(0xffffffffu, acc[i], 1);
-      const float r2 = __shfl_down_sync(0xffffffffu, acc[i], 2);
-      const float r3 = __shfl_down_sync(0xffffffffu, acc[i], 3);
-      if (g == 0) out(b, c * 8 + i, (((acc[i] + r1) + r2) + r3) * inv);
-    }
-  }
-}
-
-template <int HD>
-__global__ void __launch_bounds__(kStreamThreads, 3)
-select_stream_kernel(const __grid_constant__ StreamArgs a, const Dims D) {
-  extern __shared__ float4 sm4[];
-  float* smf = reinterpret_cast<float*>(sm4);
-  __shared__ int s_unit;
-  if (threadIdx.x == 0) s_unit = atomicAdd(&a.sync[0], 1);
-  __syncthreads();
-  const int unit = s_unit;
-#ifdef LF_TRACE
-#define LF_TR_UNIT(k)                                                                   \
-  do {                                                                                  \
-    if (g_lf_cta_trace && threadIdx.x == 0) g_lf_cta_trace[(size_t)unit * 4 + (k)] = globaltimer_ns(); \
-  } while (0)
-#else
-#define LF_TR_UNIT(k) do {} while (0)
-#endif
-  LF_TR_UNIT(0);
-  const int np = stream_parts(D), per = cdiv(D.nbpf, np);
-  const int UQ = D.H * D.Fc * np, UH = D.H * D.F * np;
-  int32_t* q_done = a.sync + 1;
-  int32_t* h_done = a.sync + 1 + D.H;
-  float* sk = smf;                                            // [kStreamBlocks][HD + 4]
-  float* sq = sk + kStreamBlocks * (HD + 4);                  // [nqb][HD]
-
-  if (unit < UQ) {                                 // ---- pooled queries
-    const int h = unit / (D.Fc * np), r = unit % (D.Fc * np);
-    const int fc = r / np, p = r % np;
-    const int b0 = p * per, b1 = min(D.nbpf, b0 + per);
-    float* dst = a.q_blk + ((size_t)h * D.nqb + (size_t)fc * D.nbpf) * HD;
-    pool_part<HD>(a.q + (size_t)fc * D.T * D.H * HD, h, b0, b1, D,
-                  [&](int b, int ch, float v) { dst[(size_t)b * HD + ch] = v; });
-    LF_TR_UNIT(1);
-    cta_signal(&q_done[h]);
-    LF_TR_UNIT(3);
-  } else if (unit < UQ + UH) {                     // ---- pooled keys and their scores
-    const int u = unit - UQ;
-    const int h = u / (D.F * np), r = u % (D.F * np);
-    const int f = r / np, p = r % np;
-    const int b0 = p * per, b1 = min(D.nbpf, b0 + per);
-    pool_part<HD>(a.k_cache + (size_t)a.hist_slots[f] * D.T * D.H * HD, h, b0, b1, D,
-                  [&](int b, int ch, float v) { sk[(b - b0) * (HD + 4) + ch] = v; });
-    LF_TR_UNIT(1);
-    if (!cta_wait_count(&q_done[h], D.Fc * np, a.wait_limit_ns)) return;
-    LF_TR_UNIT(2);
-    const float4* qsrc = reinterpret_cast<const float4*>(a.q_blk + (size_t)h * D.nqb * HD);
-    for (int i = threadIdx.x; i < D.nqb * (HD / 4); i += kStreamThreads)
-      reinterpret_cast<float4*>(sq)[i] = __ldcg(qsrc + i);
-    __syncthreads();
-    // thread task: one block x up to four query blocks (qg, qg + nqg, ...), each score one
-    // fma chain over the channels in order; consecutive threads take consecutive blocks
-    // (distinct k rows, padded pitch) of the same query blocks (broadcast q rows)
-    const int nqg = cdiv(D.nqb, 4), nb = b1 - b0, NB = D.F * D.nbpf;
-    for (int task = threadIdx.x; task < nb * nqg; task += kStreamThreads) {
-      const int bl = task % nb, qg = task / nb;
-      const float4* kr = reinterpret_cast<const float4*>(sk + bl * (HD + 4));
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const float4* qr[4];
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int qb = min(qg + v * nqg, D.nqb - 1);
-        qr[v] = reinterpret_cast<const float4*>(sq + (size_t)qb * HD);
-      }
-#pragma unroll 8
-      for (int c4 = 0; c4 < HD / 4; ++c4) {
-        const float4 k = kr[c4];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float4 q = qr[v][c4];
-          float x = acc[v];
-          x = fmaf(q.x, k.x, x); x = fmaf(q.y, k.y, x);
-          x = fmaf(q.z, k.z, x); x = fmaf(q.w, k.w, x);
-          acc[v] = x;
-        }
-      }
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int qb = qg + v * nqg;
-        if (qb < D.nqb) a.scores[((size_t)h * D.nqb + qb) * NB + (size_t)f * D.nbpf + b0 + bl] = acc[v];
-      }
-    }
-    cta_signal(&h_done[h]);
-    LF_TR_UNIT(3);
-  } else {                                         // ---- frame and block top-k, plans
-    const int u = unit - UQ - UH;
-    const int ng = cdiv(D.nqb, kFuseQb);
-    const int h = u / ng, g = u % ng;
-    if (!cta_wait_count(&h_done[h], D.F * np, a.wait_limit_ns)) return;
-    LF_TR_UNIT(2);
-    pick_group(a.scores, a.block_idx, a.plan, a.plan_cnt, D, h, g * kFuseQb, smf);
-    LF_TR_UNIT(3);
-  }
-#undef LF_TR_UNIT
 }
 
 // One-dimensional selection (no frame stage), the ablation the pages compare against
