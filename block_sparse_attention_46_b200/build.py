@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblf.so")
 SOURCES = ["lf_api.cu"]
-DEPS = ["lf_api.cu", "lf_common.cuh", "lf_select.cuh", "lf_attn.cuh", "lf_fused.cuh"]
+DEPS = ["lf_api.cu", "lf_common.cuh", "lf_select.cuh", "lf_attn.cuh", "lf_fused.cuh", "lf_fp8.cuh"]
 
 
 def nvcc() -> str:
