@@ -15,12 +15,16 @@
 //   * the key plan of a tile (sink blocks, then the sorted union of its query blocks'
 //     selected blocks, each with a bit per query block that selected it) is built by
 //     plan_kernel; a key column a row's query block did not select is masked to -inf;
-//   * warp 0 streams K tiles and warp 2 V tiles with TMA (128-byte swizzle, zero fill out
-//     of bounds), two stages each; warp 1 issues tcgen05.mma: S = Q K^T into one of two
-//     tensor-memory buffers, O += P V into a tensor-memory accumulator;
-//   * warps 4-7 run the fp32 online softmax, one query row per thread (the row's tensor
-//     memory lane): S from tensor memory, P as bf16 into shared memory, O rescaled in
-//     tensor memory only when the row maximum grows by more than 2^8 (lazy rescale);
+//   * warp 0 streams Q, then K and V tiles, with TMA (128-byte swizzle, zero fill out of
+//     bounds) into one ring of 160 KB (five 32 KB stages at d = 128) in the order the MMAs
+//     consume them; warp 1 issues tcgen05.mma: S = Q K^T into one of two tensor-memory
+//     buffers, O += P V into the tensor-memory accumulator of the softmax warpgroup that
+//     owns the key tile; warp 3 stages the tile's key plan into shared memory;
+//   * warps 4-11 are two softmax warpgroups taking alternate key tiles, each with its own
+//     fp32 online softmax state and O, one query row per thread (the row's tensor-memory
+//     lane): S from tensor memory, P as bf16 pairs written over S, O rescaled in tensor
+//     memory only when the row maximum grows by more than 2^8 (lazy rescale); the two
+//     states are merged in the epilogue;
 //   * every mbarrier wait is bounded; on expiry the CTA drains and returns with
 //     LF_ERR_TIMEOUT recorded.
 #pragma once
