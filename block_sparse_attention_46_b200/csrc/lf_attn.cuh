@@ -181,14 +181,16 @@ plan_kernel(const int32_t* __restrict__ block_idx, const int32_t* __restrict__ c
 // straddles split_pos are placed in tile-index order, so the set of split tiles (and
 // with it the rounding of their outputs) is the same on every call; the order inside
 // any other bucket changes no result.
-// (Taking heads in groups of one wave, to keep the running CTAs' history blocks within
-// L2, measured no faster on the 480p chunk.)
+// Heads are taken in groups whose keys and values fit in part of L2 (heads_per_group, chosen
+// by the host), longest first inside a group: the CTAs running at any time then read the
+// history of a few heads, which stays in L2, instead of every head's.  Keys run over
+// n_groups x cost_buckets <= kSchedBuckets buckets.
 // ---------------------------------------------------------------------------------
 constexpr int kSchedBuckets = kMaxPlan + 1;
 
 __global__ void __launch_bounds__(1024)
 schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ order, const Dims D,
-                int split_pos) {
+                int split_pos, int heads_per_group, int cost_buckets) {
   __shared__ int hist[kSchedBuckets];
   __shared__ int start[kSchedBuckets];
   __shared__ int warp_tot[32];
@@ -196,9 +198,11 @@ schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ orde
   const int nb = kSchedBuckets;
   for (int k = threadIdx.x; k < nb; k += blockDim.x) hist[k] = 0;
   __syncthreads();
-  auto key = [&](int i) {                                 // ascending key = decreasing cost
+  const int tph = tile_count(D);
+  auto key = [&](int i) {            // ascending key = head group, then decreasing cost
     const int c = plan_cnt[i];
-    return nb - 1 - min(D.B == 64 ? (c + 1) / 2 : c, nb - 1);
+    const int cost = min(D.B == 64 ? (c + 1) / 2 : c, cost_buckets - 1);
+    return (i / tph / heads_per_group) * cost_buckets + cost_buckets - 1 - cost;
   };
   for (int i = threadIdx.x; i < ntot; i += blockDim.x) atomicAdd(&hist[key(i)], 1);
   __syncthreads();
