@@ -378,6 +378,11 @@ class ChunkRun:
         self.lse = torch.empty(sh.H, self.t["q"].shape[0], device=dev)
         self.ws = torch.empty(max(lf.lf_attn_workspace_size(sh), 256), dtype=torch.uint8,
                               device=dev)
+        # the one-call path (lf_forward_chunk): its own outputs and workspace
+        self.out_f = torch.empty_like(self.t["q"])
+        self.lse_f = torch.empty_like(self.lse)
+        self.fws = torch.empty(max(lf.lf_forward_workspace_size(sh), 256), dtype=torch.uint8,
+                               device=dev)
         if e4m3:
             # the cache's keys are quantised once (model state); the queries and the current
             # chunk's keys every step, with the per-head key scales of the cache and chunk
@@ -413,6 +418,23 @@ class ChunkRun:
                                      t["v_cache"], self.ci.hist_slots, self.ci.sink_slots,
                                      self.bidx, self.out, self.lse, self.ws,
                                      cur_idx=self.cidx if self.kc > 0 else None)
+
+    def forward(self):
+        """Stages (a)-(d) of the chunk in one call; the attention takes the key plans the
+        selection's pick kernel wrote (no plan kernel) when the current chunk is dense."""
+        t = self.t
+        self.lf.lf_forward_chunk(self.sh, t["q"], t["k_cur"], t["v_cur"], t["k_cache"],
+                                 t["v_cache"], self.ci.hist_slots, self.ci.sink_slots,
+                                 self.out_f, self.lse_f, None, self.fws)
+
+    def forward_launches(self) -> int:
+        # selection (+ the current-chunk choice) | plan unless the pick wrote the plans,
+        # schedule, attn (+ merge)
+        hist = self.sh.n_hist > 0
+        sel = selection_launches(self.sh)
+        cur = (1 if hist else 2) if self.kc > 0 else 0
+        plans_ready = hist and sel == 3 and self.kc == 0
+        return sel + cur + (0 if plans_ready else 1) + 2 + (1 if tail_split(self.sh) else 0)
 
     def flops(self) -> int:
         return executed_flops(self.sh, self.bidx.cpu().numpy(),
@@ -481,16 +503,28 @@ def run_lf(args, rank, world, local_rank):
         for r in runs:
             r.attend()
 
-    # warm up eagerly, then capture each stage in a CUDA graph (removes host overhead
+    # The step is the one-call path, lf_forward_chunk per chunk (the e4m3 variant, which
+    # has no one-call entry point, uses the stage calls).  The stage breakdown (selection,
+    # attention) is timed separately through lf_select_chunk + lf_block_sparse_attn.
+    use_fwd = not args.e4m3
+
+    def fwd_stage():
+        for r in runs:
+            r.forward()
+
+    # warm up eagerly, then capture each path in a CUDA graph (removes host overhead
     # between launches; the graphs replay exactly the kernels of the C-ABI calls)
     for _ in range(3):
         sel_stage()
         att_stage()
+        if use_fwd:
+            fwd_stage()
     torch.cuda.synchronize()
     cap = torch.cuda.Stream()
     g_sel, g_att = capture(sel_stage, stream, cap), capture(att_stage, stream, cap)
+    g_fwd = capture(fwd_stage, stream, cap) if use_fwd else None
 
-    def step(record=False):
+    def stage_step(record=False):
         if record:
             ev[0].record(stream)
         g_sel.replay()
@@ -500,13 +534,26 @@ def run_lf(args, rank, world, local_rank):
         if record:
             ev[2].record(stream)
 
+    def step(record=False):
+        if not use_fwd:
+            stage_step(record)
+            return
+        if record:
+            ev[0].record(stream)
+        g_fwd.replay()
+        if record:
+            ev[1].record(stream)
+
     for _ in range(args.warmup):
         flush_l2()
         step()
+        if use_fwd:
+            flush_l2()
+            stage_step()
     torch.cuda.synchronize()
     flops = sum(r.flops() for r in runs)
     sel_bytes = sum(selection_bytes(r.sh) for r in runs if r.sh.n_hist > 0)
-    launches_per_step = sum(r.launches() for r in runs)
+    launches_per_step = sum(r.forward_launches() if use_fwd else r.launches() for r in runs)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -514,21 +561,36 @@ def run_lf(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    sel_ms, att_ms = [], []
+    step_ms, sel_ms, att_ms = [], [], []
     for _ in range(args.steps):
         flush_l2()
         step(record=True)
-        ev[2].synchronize()
-        sel_ms.append(ev[0].elapsed_time(ev[1]))
-        att_ms.append(ev[1].elapsed_time(ev[2]))
+        if use_fwd:
+            ev[1].synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[1]))
+        else:
+            ev[2].synchronize()
+            sel_ms.append(ev[0].elapsed_time(ev[1]))
+            att_ms.append(ev[1].elapsed_time(ev[2]))
+            step_ms.append(sel_ms[-1] + att_ms[-1])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     t_wall1 = time.time()
+    if use_fwd:
+        # the stage breakdown, after the timed steps (same flush, same events)
+        for _ in range(args.steps):
+            flush_l2()
+            stage_step(record=True)
+            ev[2].synchronize()
+            sel_ms.append(ev[0].elapsed_time(ev[1]))
+            att_ms.append(ev[1].elapsed_time(ev[2]))
+        torch.cuda.synchronize()
     clk = clocks.stop(t_wall0, t_wall1)
     assert lf.lf_device_status() == 0, "device status reported an error"
-
-    step_ms = [a + b for a, b in zip(sel_ms, att_ms)]
+    if use_fwd:
+        for r in runs:                 # the one-call path computes what the stage calls do
+            assert torch.equal(r.out_f, r.out), "lf_forward_chunk differs from the stage calls"
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_step = total_ms / args.steps
     if args.shard == "heads":
@@ -560,11 +622,19 @@ def run_lf(args, rank, world, local_rank):
                    "executed_gflop_per_step": flops / 1e9,
                    "selection_mb_per_step": sel_bytes / 1e6,
                    "ms_per_chunk": ms_step / n_chunks,
+                   "step_api": ("lf_forward_chunk per chunk (the attention takes the key plans "
+                                "the selection's pick kernel wrote)") if use_fwd else
+                               "lf_select_chunk (+ lf_select_current) + quantisation + "
+                               "lf_block_sparse_attn_e4m3",
                    "ms_selection_abc": sel_mean, "ms_attention_d": att_mean,
+                   "stage_breakdown": "ms_selection_abc and ms_attention_d timed separately "
+                                      "through lf_select_chunk and lf_block_sparse_attn",
                    "selection_share": sel_mean / (sel_mean + att_mean)},
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": att_tflops / pk["bf16_tflops"],
-                     "traffic": profiled_traffic(args.config) if n_chunks == 1 else None,
+                     # the committed DRAM figures are the bf16 kernel's
+                     "traffic": profiled_traffic(args.config)
+                     if n_chunks == 1 and not args.e4m3 else None,
                      "kernel": "stage (d): plan + schedule + attn_kernel + merge (lf_block_sparse_attn)",
                      "peak_source": f"{src} bf16_tflops (burst)"},
         "e2e": e2e,
