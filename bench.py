@@ -429,21 +429,20 @@ class ChunkRun:
 
     def forward_launches(self) -> int:
         # selection (+ the current-chunk choice) | plan unless the pick wrote the plans,
-        # schedule, attn (+ merge)
+        # attn (+ merge)
         hist = self.sh.n_hist > 0
         sel = selection_launches(self.sh)
         cur = (1 if hist else 2) if self.kc > 0 else 0
         plans_ready = hist and sel == 3 and self.kc == 0
-        return sel + cur + (0 if plans_ready else 1) + 2 + (1 if tail_split(self.sh) else 0)
+        return sel + cur + (0 if plans_ready else 1) + 1 + (1 if tail_split(self.sh) else 0)
 
     def flops(self) -> int:
         return executed_flops(self.sh, self.bidx.cpu().numpy(),
                               self.cidx.cpu().numpy() if self.kc > 0 else None)
 
     def launches(self) -> int:
-        # selection kernels (+ current-chunk pooling and choice) | plan, schedule, attn
-        # (+ merge)
-        return selection_launches(self.sh) + (2 if self.kc > 0 else 0) + 3 + \
+        # selection kernels (+ current-chunk pooling and choice) | plan, attn (+ merge)
+        return selection_launches(self.sh) + (2 if self.kc > 0 else 0) + 2 + \
             (1 if tail_split(self.sh) else 0) + (2 if self.e4m3 else 0)
 
 
@@ -635,7 +634,7 @@ def run_lf(args, rank, world, local_rank):
                      # the committed DRAM figures are the bf16 kernel's
                      "traffic": profiled_traffic(args.config)
                      if n_chunks == 1 and not args.e4m3 else None,
-                     "kernel": "stage (d): plan + schedule + attn_kernel + merge (lf_block_sparse_attn)",
+                     "kernel": "stage (d): plan + attn_kernel + merge (lf_block_sparse_attn)",
                      "peak_source": f"{src} bf16_tflops (burst)"},
         "e2e": e2e,
         "incremental_compression": inc,

@@ -248,29 +248,9 @@ Split make_split(const Dims& D, int n_sm) {
   return sp;
 }
 
-// Launch order of the attention tiles: heads in groups whose keys and values (sinks,
-// history, current chunk) take at most kL2GroupBytes, so that the history the running CTAs
-// read stays in L2; by decreasing cost inside a group.  cost_buckets covers every tile's
-// cost (key tiles); groups x buckets must fit the scheduler's kSchedBuckets.
-constexpr double kL2GroupBytes = 64.0 * 1024 * 1024;
-void schedule_groups(const Dims& D, int* heads_per_group, int* cost_buckets) {
-  const int per = D.B == 64 ? 2 : 1;
-  *cost_buckets = lf::cdiv(D.ncur, 128) + lf::cdiv(lf::plan_stride(D), per) + 1;
-  const double head_bytes = ((double)(D.S + D.F) * D.T + D.ncur) * D.d * 2.0 * 2.0;
-  int g = (int)(kL2GroupBytes / head_bytes);
-  g = g < 1 ? 1 : (g > D.H ? D.H : g);
-  while (g < D.H && (long long)lf::cdiv(D.H, g) * *cost_buckets > lf::kSchedBuckets) ++g;
-  if ((long long)lf::cdiv(D.H, g) * *cost_buckets > lf::kSchedBuckets) {   // one group
-    g = D.H;
-    if (*cost_buckets > lf::kSchedBuckets) *cost_buckets = lf::kSchedBuckets;
-  }
-  *heads_per_group = g;
-}
-
 struct AttnWs {
   uint32_t* plan;
   int32_t* plan_cnt;
-  int32_t* order;
   float* part_o;
   float* part_ml;
   size_t bytes;
@@ -286,7 +266,6 @@ AttnWs carve_attn(const Dims& D, void* base, int n_sm) {
   const size_t units = n_sm > 0 ? (size_t)n_sm : 0;
   w.plan = reinterpret_cast<uint32_t*>(take(nt * lf::plan_stride(D) * sizeof(uint32_t)));
   w.plan_cnt = reinterpret_cast<int32_t*>(take(nt * sizeof(int32_t)));
-  w.order = reinterpret_cast<int32_t*>(take(nt * sizeof(int32_t)));
   w.part_o = reinterpret_cast<float*>(take(units * 128 * D.d * sizeof(float)));
   w.part_ml = reinterpret_cast<float*>(take(units * 2 * 128 * sizeof(float)));
   w.bytes = off;
@@ -317,16 +296,11 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   const int n_sm = sm_count();
   if (n_sm <= 0) return LF_ERR_CUDA;
   const AttnWs w = carve_attn(D, workspace, n_sm);
-  // key plans (unless the fused selection already wrote them), then the launch order
+  // key plans (unless the fused selection already wrote them)
   if (!plans_ready)
     lf::plan_kernel<<<dim3(lf::cdiv(lf::tile_count(D), lf::kPlanWarps), D.H), lf::kPlanWarps * 32, 0, st>>>(
         D.F > 0 ? block_idx : nullptr, D.kc > 0 ? cur_idx : nullptr, w.plan, w.plan_cnt, D);
   const Split sp = make_split(D, n_sm);
-  int hpg, cb;
-  schedule_groups(D, &hpg, &cb);
-  lf::schedule_kernel<<<1, 1024, 0, st>>>(w.plan_cnt, w.order, D,
-                                          sp.n_tail > 0 ? sp.n_whole : lf::tile_count(D) * D.H,
-                                          hpg, cb);
   int rc = cuda_status(cudaGetLastError());
   if (rc != LF_OK) return rc;
 
@@ -356,7 +330,6 @@ int launch_attn(const Dims& D, const void* q, const void* k_cur, const void* v_c
   }
   p.plan = w.plan;
   p.plan_cnt = w.plan_cnt;
-  p.order = w.order;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.tiles_per_head = lf::tile_count(D);

@@ -173,108 +173,6 @@ plan_kernel(const int32_t* __restrict__ block_idx, const int32_t* __restrict__ c
   }
 }
 
-// ---------------------------------------------------------------------------------
-// Launch order of the tiles: longest first (list scheduling by decreasing cost, so the
-// last CTAs to start are the cheapest).  Cost = key tiles = dense tiles + sparse tiles;
-// a counting sort over the cost; one CTA of 1024 threads.  Positions from split_pos on
-// are the tail tiles that run split into pieces: the tiles of the cost bucket that
-// straddles split_pos are placed in tile-index order, so the set of split tiles (and
-// with it the rounding of their outputs) is the same on every call; the order inside
-// any other bucket changes no result.
-// Heads are taken in groups whose keys and values fit in part of L2 (heads_per_group, chosen
-// by the host), longest first inside a group: the CTAs running at any time then read the
-// history of a few heads, which stays in L2, instead of every head's.  Keys run over
-// n_groups x cost_buckets <= kSchedBuckets buckets.
-// ---------------------------------------------------------------------------------
-constexpr int kSchedBuckets = kMaxPlan + 1;
-
-__global__ void __launch_bounds__(1024)
-schedule_kernel(const int32_t* __restrict__ plan_cnt, int32_t* __restrict__ order, const Dims D,
-                int split_pos, int heads_per_group, int cost_buckets) {
-  __shared__ int hist[kSchedBuckets];
-  __shared__ int start[kSchedBuckets];
-  __shared__ int warp_tot[32];
-  const int ntot = tile_count(D) * D.H;
-  const int nb = kSchedBuckets;
-  for (int k = threadIdx.x; k < nb; k += blockDim.x) hist[k] = 0;
-  __syncthreads();
-  const int tph = tile_count(D);
-  auto key = [&](int i) {            // ascending key = head group, then decreasing cost
-    const int c = plan_cnt[i];
-    const int cost = min(D.B == 64 ? (c + 1) / 2 : c, cost_buckets - 1);
-    return (i / tph / heads_per_group) * cost_buckets + cost_buckets - 1 - cost;
-  };
-  for (int i = threadIdx.x; i < ntot; i += blockDim.x) atomicAdd(&hist[key(i)], 1);
-  __syncthreads();
-  // exclusive scan of the histogram in key order
-  const int per = (nb + blockDim.x - 1) / blockDim.x;     // buckets per thread
-  int local = 0;
-  for (int q = 0; q < per; ++q) {
-    const int k = threadIdx.x * per + q;
-    if (k < nb) local += hist[k];
-  }
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int incl = local;
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += y;
-  }
-  if (lane == 31) warp_tot[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    int v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, v, off);
-      if (lane >= off) v += y;
-    }
-    warp_tot[lane] = v;                                  // inclusive over warps
-  }
-  __syncthreads();
-  int run = (w > 0 ? warp_tot[w - 1] : 0) + incl - local;
-  for (int q = 0; q < per; ++q) {
-    const int k = threadIdx.x * per + q;
-    if (k < nb) {
-      start[k] = run;
-      run += hist[k];
-    }
-  }
-  // the bucket holding position split_pos (if the tail is split) goes in index order
-  __shared__ int kb_split, split_next, wpre[32];
-  if (threadIdx.x == 0) kb_split = -1;
-  __syncthreads();
-  for (int k = threadIdx.x; k < nb; k += blockDim.x)
-    if (start[k] <= split_pos && split_pos < start[k] + hist[k]) {
-      kb_split = k;
-      split_next = start[k];
-    }
-  __syncthreads();
-  for (int base = 0; base < ntot; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    const int k = i < ntot ? key(i) : -1;
-    const bool ordered = i < ntot && k == kb_split;
-    const uint32_t bal = __ballot_sync(0xffffffffu, ordered);
-    if (lane == 0) wpre[w] = __popc(bal);
-    __syncthreads();
-    if (w == 0) {                                  // exclusive prefix over the warps
-      const int x = lane < (int)(blockDim.x >> 5) ? wpre[lane] : 0;
-      int inc = x;
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, inc, off);
-        if (lane >= off) inc += y;
-      }
-      wpre[lane] = inc - x;
-      if (lane == 31) warp_tot[0] = inc;           // ordered tiles in this chunk
-    }
-    __syncthreads();
-    if (ordered)
-      order[split_next + wpre[w] + __popc(bal & ((1u << lane) - 1u))] = i;
-    else if (i < ntot)
-      order[atomicAdd(&start[k], 1)] = i;
-    __syncthreads();
-    if (threadIdx.x == 0) split_next += warp_tot[0];
-    __syncthreads();
-  }
-}
 
 // ---------------------------------------------------------------------------------
 // Attention kernel
@@ -287,7 +185,6 @@ struct AttnParams {
   CUtensorMap tm_vh;
   const uint32_t* plan;
   const int32_t* plan_cnt;
-  const int32_t* order;  // launch position -> tile (longest first)
   __nv_bfloat16* out;  // [ncur, H, d]
   float* lse;          // [H, ncur] or null
   // work decomposition: CTAs [0, n_whole) take tiles whole; the remaining tiles (the last
@@ -394,7 +291,9 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     piece = (blockIdx.x - P.n_whole) % P.pieces;
     pos = P.n_whole + tail;
   }
-  const int tile = P.order[pos];
+  // tiles in index order (head-major): the CTAs running at any time read the history of
+  // a few heads, which stays in L2; the last partial wave is split (see n_whole)
+  const int tile = pos;
   const int h = tile / P.tiles_per_head, t = tile % P.tiles_per_head;
 
   // query blocks of this tile
@@ -828,7 +727,7 @@ constexpr int kMaxPieces = 16;     // key ranges a tail tile is split into, at m
 __global__ void __launch_bounds__(256)
 merge_kernel(const AttnParams P, const Dims D, int HD) {
   const int tail = blockIdx.x;
-  const int tile = P.order[P.n_whole + tail];
+  const int tile = P.n_whole + tail;
   const int h = tile / P.tiles_per_head, t = tile % P.tiles_per_head;
   const int qbA = D.B == 64 ? 2 * t : t;
   const int qbB = (D.B == 64 && 2 * t + 1 < D.nqb) ? 2 * t + 1 : -1;

@@ -117,7 +117,7 @@ def test_clock_summary_from_fake_rows():
 def test_forward_launch_counts():
     """Kernels one lf_forward_chunk call launches (the benchmark's gpu_launches claim):
     selection, the current-chunk choice when it is sparse, plan_kernel unless the pick
-    kernel wrote the plans, schedule, attention, and merge when the tail is split."""
+    kernel wrote the plans, attention, and merge when the tail is split."""
     from dataclasses import replace
     import lf_workloads as W
 
@@ -125,12 +125,12 @@ def test_forward_launch_counts():
         def __init__(self, sh, kc):
             self.sh, self.kc = sh, kc
     p480 = W.p480_shape()
-    assert bench.ChunkRun.forward_launches(Run(p480, 0)) == 3 + 2 + 1       # tail split
-    assert bench.ChunkRun.forward_launches(Run(W.large_shape(), 0)) == 3 + 2
+    assert bench.ChunkRun.forward_launches(Run(p480, 0)) == 3 + 1 + 1       # tail split
+    assert bench.ChunkRun.forward_launches(Run(W.large_shape(), 0)) == 3 + 1
     # sparse current chunk: its pooling shares the selection's launch, then its choice and
     # plan_kernel
-    assert bench.ChunkRun.forward_launches(Run(replace(p480, k_c=15), 15)) == 3 + 1 + 1 + 2 + 1
+    assert bench.ChunkRun.forward_launches(Run(replace(p480, k_c=15), 15)) == 3 + 1 + 1 + 1 + 1
     # first chunk (no history): query/current pooling and the choice, plan_kernel
     first = replace(p480, n_hist=0, k_c=15)
     assert bench.ChunkRun.forward_launches(Run(first, 15)) == \
-        2 + 1 + 2 + (1 if bench.tail_split(first) else 0)
+        2 + 1 + 1 + (1 if bench.tail_split(first) else 0)
