@@ -313,6 +313,69 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     n_iter = (int)((long long)(piece + 1) * n_tile / P.pieces) - j0;
   }
 
+  // TMA loads of Q, and of ring position q (tile l, a key tile when isK) armed on its slot's
+  // full barrier; sparse tiles read the staged key plan, dense ones (j < n_dense) do not
+  auto load_q = [&]() {
+    if (F8) {
+      mbar_arrive_expect_tx(&bars[kBarQ], 128 * HD);         // e4m3: one byte per element
+      uint8_t* dst = smem + L::kQ;
+      tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD, tokA);
+      tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD, BLK == 64 ? tokB : tokA + 64);
+    } else {
+      mbar_arrive_expect_tx(&bars[kBarQ], L::kQBytes);
+      for (int c = 0; c < L::NH; ++c) {
+        uint8_t* dst = smem + L::kQ + c * L::kRegion;
+        tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD + c * 64, tokA);
+        tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD + c * 64,
+                    BLK == 64 ? tokB : tokA + 64);
+      }
+    }
+  };
+  auto load_pos = [&](int q, bool isK, int l) {
+    uint64_t* full = &bars[kBarRing];
+    const int slot = q % L::kSlots;
+    const int j = j0 + l;
+    LF_TR(isK ? 0 : 1, l);
+    const bool f8 = F8 && isK;                     // an e4m3 key tile: one 16 KB region
+    const int nreg = f8 ? 1 : L::NH;
+    const int xcol = f8 ? h * HD : 0;               // x coordinate base: bytes / elements
+    mbar_arrive_expect_tx(&full[slot], f8 ? 128 * HD : L::kStageBytes);
+    uint8_t* st = smem + L::kRing + slot * L::kStageBytes;
+    const CUtensorMap* tm_cur = isK ? &P.tm_kc : &P.tm_vc;
+    const CUtensorMap* tm_hist = isK ? &P.tm_kh : &P.tm_vh;
+    for (int box = 0; box < 2; ++box) {
+      if (j < n_dense) {
+        const int row = j * 128 + box * 64;
+        for (int c = 0; c < nreg; ++c)
+          tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
+                      f8 ? xcol : h * HD + c * 64, row);
+      } else {
+        const int u = j - n_dense;
+        int slot_id = 0, tok = 0;
+        int p = -1;                                    // -1: padding past the plan's end
+        const int e = BLK == 64 ? 2 * u + box : u;
+        if (e < cnt) {
+          const uint32_t pe = s_plan[e];
+          p = (int)(pe >> 16);
+          tok = (int)((pe >> 4) & 0xFFFu) * BLK + (BLK == 64 ? 0 : box * 64);
+          if (p < D.S + D.F) slot_id = P.slots[p];
+        }
+        if (p < 0 || p >= D.S + D.F) {
+          // a block of the current chunk (2-D map), or padding: rows from ncur on are
+          // out of bounds and read as zero (the columns are masked anyway)
+          const int row = p < 0 ? D.ncur : (p - D.S - D.F) * D.T + tok;
+          for (int c = 0; c < nreg; ++c)
+            tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
+                        f8 ? xcol : h * HD + c * 64, row);
+        } else {
+          for (int c = 0; c < nreg; ++c)
+            tma_load_3d(st + c * L::kRegion + box * 64 * 128, tm_hist, &full[slot],
+                        f8 ? xcol : h * HD + c * 64, tok, slot_id);
+        }
+      }
+    }
+  };
+  int pre = 0;                                     // ring positions loaded in the set-up
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarQ], 1);
     for (int s = 0; s < 2; ++s) {
@@ -324,6 +387,12 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     mbar_init(&bars[kBarDone], 1);
     *s_abort = 0;
     fence_mbar_init();
+    // Q and the first key tiles when they are dense (no key plan needed) go out now, so
+    // their latency overlaps the tensor-memory allocation and the plan staging
+    prefetch_tmap(&P.tm_q); prefetch_tmap(&P.tm_kc); prefetch_tmap(&P.tm_kh);
+    prefetch_tmap(&P.tm_vc); prefetch_tmap(&P.tm_vh);
+    if (!(P.debug_stall && blockIdx.x == 0)) load_q();
+    for (; pre < 2 && pre < n_iter && j0 + pre < n_dense; ++pre) load_pos(pre, true, pre);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, L::kTmemCols);
@@ -335,10 +404,6 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     LF_TR_CTA(3, n_iter);
   }
   if (warp == 3) stage_words(s_plan, P.plan + (size_t)tile * plan_stride(D), cnt, lane, 32);
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&P.tm_q); prefetch_tmap(&P.tm_kc); prefetch_tmap(&P.tm_kh);
-    prefetch_tmap(&P.tm_vc); prefetch_tmap(&P.tm_vh);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -350,22 +415,8 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   if (warp == 0 && lane == 0) {
     uint64_t* full = &bars[kBarRing];
     uint64_t* empty = &bars[kBarRing + L::kSlots];
-    if (F8 && !(P.debug_stall && blockIdx.x == 0)) {
-      mbar_arrive_expect_tx(&bars[kBarQ], 128 * HD);         // e4m3: one byte per element
-      uint8_t* dst = smem + L::kQ;
-      tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD, tokA);
-      tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD, BLK == 64 ? tokB : tokA + 64);
-    } else if (!(P.debug_stall && blockIdx.x == 0)) {
-      mbar_arrive_expect_tx(&bars[kBarQ], L::kQBytes);
-      for (int c = 0; c < L::NH; ++c) {
-        uint8_t* dst = smem + L::kQ + c * L::kRegion;
-        tma_load_2d(dst, &P.tm_q, &bars[kBarQ], h * HD + c * 64, tokA);
-        tma_load_2d(dst + 64 * 128, &P.tm_q, &bars[kBarQ], h * HD + c * 64,
-                    BLK == 64 ? tokB : tokA + 64);
-      }
-    }
     const int n_pos = 2 * n_iter + 1;               // V of the last tile sits at 2n
-    int q = 0;
+    int q = pre;                                    // positions loaded in the set-up
     for (; q < n_pos; ++q) {
       bool isK;
       const int l = ring_tile(q, isK);
@@ -373,46 +424,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       const int rnd = q / L::kSlots;
       if (isK && l >= n_iter) continue;            // no slot used, nothing to load
       if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort, P.wait_limit_ns)) break;
-      const int j = j0 + l;
-      LF_TR(isK ? 0 : 1, l);
-      const bool f8 = F8 && isK;                     // an e4m3 key tile: one 16 KB region
-      const int nreg = f8 ? 1 : L::NH;
-      const int xcol = f8 ? h * HD : 0;               // x coordinate base: bytes / elements
-      mbar_arrive_expect_tx(&full[slot], f8 ? 128 * HD : L::kStageBytes);
-      uint8_t* st = smem + L::kRing + slot * L::kStageBytes;
-      const CUtensorMap* tm_cur = isK ? &P.tm_kc : &P.tm_vc;
-      const CUtensorMap* tm_hist = isK ? &P.tm_kh : &P.tm_vh;
-      for (int box = 0; box < 2; ++box) {
-        if (j < n_dense) {
-          const int row = j * 128 + box * 64;
-          for (int c = 0; c < nreg; ++c)
-            tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
-                        f8 ? xcol : h * HD + c * 64, row);
-        } else {
-          const int u = j - n_dense;
-          int slot_id = 0, tok = 0;
-          int p = -1;                                    // -1: padding past the plan's end
-          const int e = BLK == 64 ? 2 * u + box : u;
-          if (e < cnt) {
-            const uint32_t pe = s_plan[e];
-            p = (int)(pe >> 16);
-            tok = (int)((pe >> 4) & 0xFFFu) * BLK + (BLK == 64 ? 0 : box * 64);
-            if (p < D.S + D.F) slot_id = P.slots[p];
-          }
-          if (p < 0 || p >= D.S + D.F) {
-            // a block of the current chunk (2-D map), or padding: rows from ncur on are
-            // out of bounds and read as zero (the columns are masked anyway)
-            const int row = p < 0 ? D.ncur : (p - D.S - D.F) * D.T + tok;
-            for (int c = 0; c < nreg; ++c)
-              tma_load_2d(st + c * L::kRegion + box * 64 * 128, tm_cur, &full[slot],
-                          f8 ? xcol : h * HD + c * 64, row);
-          } else {
-            for (int c = 0; c < nreg; ++c)
-              tma_load_3d(st + c * L::kRegion + box * 64 * 128, tm_hist, &full[slot],
-                          f8 ? xcol : h * HD + c * 64, tok, slot_id);
-          }
-        }
-      }
+      load_pos(q, isK, l);
     }
     // drain: every load issued must land before the CTA may exit (the last kSlots
     // positions hold the only loads that nobody may have waited for)
