@@ -38,11 +38,12 @@ struct PoolArgs {
 constexpr int kPoolCols = 64;       // 8-channel groups per CTA (threads per token group)
 constexpr int kPoolGroups = 4;      // token groups per CTA: a block's tokens split in 4 runs
 constexpr int kPoolThreads = kPoolCols * kPoolGroups;
-constexpr int kPoolUnroll = 16;
+constexpr int kPoolUnroll = 8;     // 16-byte loads in flight per thread
 
 // Thread (token group g, column group c): sums its run of the block's tokens in token order
-// (16-byte loads, up to 16 in flight); the four runs are then added in run order.
-__global__ void __launch_bounds__(kPoolThreads, 2)
+// (16-byte loads, up to kPoolUnroll in flight; four CTAs per SM keep ~128 KB in flight per
+// SM); the four runs are then added in run order.
+__global__ void __launch_bounds__(kPoolThreads, 4)
 pool_blocks_kernel(const __grid_constant__ PoolArgs a, const Dims D) {
   __shared__ float part[kPoolGroups][kPoolCols][8];
   const int unit = blockIdx.x;
