@@ -18,13 +18,14 @@
 //   * warp 0 streams Q, then K and V tiles, with TMA (128-byte swizzle, zero fill out of
 //     bounds) into one ring of 160 KB (five 32 KB stages at d = 128) in the order the MMAs
 //     consume them; warp 1 issues tcgen05.mma: S = Q K^T into one of two tensor-memory
-//     buffers, O += P V into the tensor-memory accumulator of the softmax warpgroup that
-//     owns the key tile; warp 3 stages the tile's key plan into shared memory;
-//   * warps 4-11 are two softmax warpgroups taking alternate key tiles, each with its own
-//     fp32 online softmax state and O, one query row per thread (the row's tensor-memory
-//     lane): S from tensor memory, P as bf16 pairs written over S, O rescaled in tensor
-//     memory only when the row maximum grows by more than 2^8 (lazy rescale); the two
-//     states are merged in the epilogue;
+//     buffers (S of tile l+1 is computed while the softmax works on tile l), and per
+//     softmax warpgroup O_w += P_w V_w over that warpgroup's 64 keys of the tile; warp 3
+//     stages the tile's key plan into shared memory;
+//   * warps 4-11 are two softmax warpgroups; warpgroup w takes keys [64w, 64w + 64) of
+//     every key tile and keeps its own fp32 online softmax state and O_w over them, one
+//     query row per thread (the row's tensor-memory lane): S from tensor memory, P as bf16
+//     pairs written over S, O_w rescaled in tensor memory only when its row maximum grows
+//     by more than 2^8 (lazy rescale); the two states are merged in the epilogue;
 //   * every mbarrier wait is bounded; on expiry the CTA drains and returns with
 //     LF_ERR_TIMEOUT recorded.
 #pragma once
@@ -203,6 +204,11 @@ struct AttnParams {
   int slots[LF_MAX_FRAMES];   // cache slot of frame position p (sinks, then history)
 };
 
+// barrier indices: ring full/empty barriers follow these
+// P barriers: kBarPFull + 2 * buffer + warpgroup (keys 0-63, 64-127 of the tile)
+// kBarPVLast: completion of the PVs of the last tile but one (committed once)
+enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 7, kBarPVLast = 8, kBarRing = 9 };
+
 template <int HD>
 struct AttnLayout {
   static constexpr int NH = HD / 64;                 // 64-column halves of the head dim
@@ -216,19 +222,16 @@ struct AttnLayout {
   static constexpr int kPlan = kRing + kSlots * kStageBytes;
   static constexpr int kRed = kPlan + kMaxPlan * 4;  // per-row (m, l) of both warpgroups
   static constexpr int kBar = kRed + 2 * 2 * 128 * 4;
-  static constexpr int kNumBars = 2 * kSlots + 8;
+  static constexpr int kNumBars = 2 * kSlots + kBarRing;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;       // slack for 1024-byte alignment
   // tensor-memory columns: two O accumulators (one per softmax warpgroup), two S buffers;
-  // P (bf16 pairs) overwrites the first 64 columns of the S buffer it was computed from
+  // warpgroup w's P (bf16 pairs) overwrites columns [64w, 64w + 32) of the S buffer it was
+  // computed from
   static constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS0 = 256, kColS1 = 384,
                             kTmemCols = 512;
 };
-
-// barrier indices: ring full/empty barriers follow these
-// P barriers: kBarPFull + 2 * buffer + half (keys 0-63, 64-127)
-enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 7, kBarRing = 8 };
 
 // position of a tile in the ring's load order: K0, K1, V0, K2, V1, K3, V2, ...
 __device__ __forceinline__ int ring_pos_k(int j) { return j < 2 ? j : 2 * j - 1; }
@@ -256,7 +259,7 @@ __device__ __forceinline__ float row_max(const float* v) {
   return fmaxf(fmax3f(m[0], m[1], m[2]), fmax3f(fmax3f(m[3], m[4], m[5]), m[6], m[7]));
 }
 
-constexpr int kSoftmaxWarps = 8;          // two warpgroups, alternate key tiles
+constexpr int kSoftmaxWarps = 8;          // two warpgroups, one 64-key half of every tile each
 // Register split: launched at 168 per thread (384 threads); the load/MMA warpgroup gives
 // registers to the two softmax warpgroups: 128 x 72 + 256 x 216 <= 384 x 168.
 constexpr int kLaunchRegs = 168, kLowRegs = 72, kHighRegs = 216;
@@ -385,6 +388,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     }
     for (int q = 0; q < 2 * L::kSlots; ++q) mbar_init(&bars[kBarRing + q], 1);
     mbar_init(&bars[kBarDone], 1);
+    mbar_init(&bars[kBarPVLast], 1);
     *s_abort = 0;
     fence_mbar_init();
     // Q and the first key tiles when they are dense (no key plan needed) go out now, so
@@ -435,9 +439,10 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     }
   }
   // -------------------------------------------------------------- MMA issuer
-  // Order: S0, S1, then for each l: PV_l (O_{l&1} += P_l V_l), S_{l+2} into the S buffer
-  // P_l was read from.  tcgen05.mma runs in issue order, so S_{l+2} overwrites P_l only
-  // after PV_l has consumed it, and the completion of S_{l+2} implies that of PV_l.
+  // Order: S0, S1, then for each l: PV_l of warpgroup 0 and of warpgroup 1 (O_w += P_w V_w,
+  // the warpgroup's 64 keys of tile l), S_{l+2} into the S buffer P_l was read from.
+  // tcgen05.mma runs in issue order, so S_{l+2} overwrites P_l only after both PVs have
+  // consumed it, and the completion of S_{l+1} implies that of PV_{l-1}.
   else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, 0, 1);
@@ -480,26 +485,26 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort, P.wait_limit_ns);
       LF_TR(4, l);
       const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
-      const uint32_t o_tmem = tmem + (s ? L::kColO1 : L::kColO0);
-      // P arrives in two halves (keys 0-63, 64-127); each half's four MMAs go as soon
-      // as it is written
-      for (int hf = 0; ok && hf < 2; ++hf) {
-        ok = mbar_wait(&bars[kBarPFull + 2 * s + hf], (l >> 1) & 1, s_abort, P.wait_limit_ns);
+      // each warpgroup's P (its 64 keys) goes into its own O as soon as it is written
+      for (int wg = 0; ok && wg < 2; ++wg) {
+        ok = mbar_wait(&bars[kBarPFull + 2 * s + wg], (l >> 1) & 1, s_abort, P.wait_limit_ns);
         if (!ok) break;
-        if (hf == 0) LF_TR(5, l);
+        if (wg == 0) LF_TR(5, l);
         tc_fence_after();
+        const uint32_t o_tmem = tmem + (wg ? L::kColO1 : L::kColO0);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {        // 16 keys per MMA, 8 P columns each
-          const int ks = hf * 4 + k4;
-          mma_bf16_ts(o_tmem, p_tmem + ks * 8,
+          const int ks = wg * 4 + k4;           // 16-key step within the V tile
+          mma_bf16_ts(o_tmem, p_tmem + wg * 64 + k4 * 8,
                       smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
                                       L::kRegion, 1024),
-                      idesc_pv, (l >= 2 || ks > 0) ? 1u : 0u);
+                      idesc_pv, (l > 0 || k4 > 0) ? 1u : 0u);
         }
       }
       if (!ok) break;
       mma_commit(&empty[vslot]);
       if (l + 2 < n_iter) ok = issue_s(l + 2);
+      else if (l + 2 == n_iter) mma_commit(&bars[kBarPVLast]);   // no S_{l+2} to imply it
     }
     // completion of everything issued: epilogue may read O, tensor memory may be freed
     mma_commit(&bars[kBarDone]);
@@ -508,11 +513,10 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   regs_inc<kHighRegs>();
   // -------------------------------------------------------------- softmax + epilogue
   {
-    const int wg = (warp - 4) >> 2;                        // handles local tiles wg, wg+2, ...
+    const int wg = (warp - 4) >> 2;                        // keys [64 wg, 64 wg + 64) of each tile
     const int r = (threadIdx.x - 128) & 127;               // query row = TMEM lane
     const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t row_bit = (BLK == 64 && r >= 64) ? 2u : 1u;
-    const uint32_t s_col = wg ? L::kColS1 : L::kColS0;
     const uint32_t o_col = wg ? L::kColO1 : L::kColO0;
     // scale * log2(e), times the row's query scale and the head's key scale for e4m3 Q/K
     float c = D.scale * 1.4426950408889634f;
@@ -524,66 +528,52 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int n_mine = 0;                                        // PVs into this group's O
-    for (int l = wg; l < n_iter; l += 2, ++n_mine) {
-      const int j = j0 + l;
+    for (int l = 0; l < n_iter; ++l) {
+      const int j = j0 + l, sb = l & 1;
+      const uint32_t s_col = (sb ? L::kColS1 : L::kColS0) + wg * 64;
       if (threadIdx.x == 128) LF_TR(6, l);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + wg], (l >> 1) & 1, s_abort, P.wait_limit_ns)) && ok;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + sb], (l >> 1) & 1, s_abort, P.wait_limit_ns)) && ok;
       if (threadIdx.x == 128) LF_TR(7, l);
       tc_fence_after();
-      float sv[128];
+      float sv[64];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld32(t_row + s_col + ch * 32, sv + ch * 32);
+      for (int ch = 0; ch < 2; ++ch) tmem_ld32(t_row + s_col + ch * 32, sv + ch * 32);
       tmem_ld_wait();
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) reg_fence32(sv + ch * 32);
+      for (int ch = 0; ch < 2; ++ch) reg_fence32(sv + ch * 32);
       if (threadIdx.x == 128) LF_TR(8, l);
 
-      // valid key columns of this row: [0, v0) and [64, 64 + v1)
-      int v0, v1;
+      // valid key columns [0, v) of this warpgroup's 64 (warp-uniform: a warp's 32 rows
+      // belong to one query block)
+      int v;
       if (j < n_dense) {
-        const int n = min(128, D.ncur - j * 128);
-        v0 = min(64, n);
-        v1 = max(0, n - 64);
+        v = max(0, min(64, D.ncur - j * 128 - wg * 64));
       } else {
         const int u = j - n_dense;
         if (BLK == 64) {
-          v0 = v1 = 0;
-          if (2 * u < cnt) {
-            const uint32_t e = s_plan[2 * u];
-            if (e & row_bit) v0 = block_len(D, (e >> 4) & 0xFFF);
-          }
-          if (2 * u + 1 < cnt) {
-            const uint32_t e = s_plan[2 * u + 1];
-            if (e & row_bit) v1 = block_len(D, (e >> 4) & 0xFFF);
+          const int e = 2 * u + wg;
+          v = 0;
+          if (e < cnt) {
+            const uint32_t pe = s_plan[e];
+            if (pe & row_bit) v = block_len(D, (pe >> 4) & 0xFFF);
           }
         } else {
-          const uint32_t e = s_plan[u];
-          const int len = (e & row_bit) ? block_len(D, (e >> 4) & 0xFFF) : 0;
-          v0 = min(64, len);
-          v1 = max(0, len - 64);
+          const uint32_t pe = s_plan[u];
+          const int len = (pe & row_bit) ? block_len(D, (pe >> 4) & 0xFFF) : 0;
+          v = max(0, min(64, len - wg * 64));
         }
       }
-      // row maximum over the valid columns (v0, v1 are warp-uniform: a warp's 32 rows
-      // belong to one query block).  A half that is wholly valid or wholly masked needs no
-      // per-column masking (a wholly masked half is left out of the maximum and skips its
-      // exponentials below); only a partly valid half (a short last block of a frame, or
-      // the end of the current chunk) is masked column by column.
+      // row maximum over the valid columns: a wholly valid half needs no masking, a wholly
+      // masked one is left out (and skips its exponentials below); only a partly valid half
+      // (a short last block of a frame, or the end of the current chunk) is masked
       float m_raw;
-      const bool full0 = v0 == 64, full1 = v1 == 64;
-      if ((v0 != 0 && !full0) || (v1 != 0 && !full1)) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          if (i >= v0) sv[i] = -INFINITY;
-          if (i >= v1) sv[64 + i] = -INFINITY;
-        }
-        m_raw = row_max<128>(sv);
-      } else if (full0 && full1) {
-        m_raw = row_max<128>(sv);
-      } else if (full0) {
+      if (v == 64) {
         m_raw = row_max<64>(sv);
-      } else if (full1) {
-        m_raw = row_max<64>(sv + 64);
+      } else if (v > 0) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i >= v) sv[i] = -INFINITY;
+        m_raw = row_max<64>(sv);
       } else {
         m_raw = -INFINITY;
       }
@@ -591,8 +581,15 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       float m_new = m_run;
       bool resc = false;
       if (m_tile > m_run + 8.0f) { m_new = m_tile; resc = true; }
-      // lazy rescale of this group's O: its previous PV (PV_{l-2}) completed before S_l did
-      if (n_mine > 0 && __any_sync(0xffffffffu, resc)) {
+      // lazy rescale of this group's O.  Its last PV (PV_{l-1}) was issued after S_l, so it
+      // is waited for: it completed before S_{l+1} did, or, when l is the last tile, before
+      // the commit that follows it.
+      if (l > 0 && __any_sync(0xffffffffu, resc)) {
+        const bool w = l + 1 < n_iter
+            ? mbar_wait(&bars[kBarSFull + (sb ^ 1)], ((l + 1) >> 1) & 1, s_abort, P.wait_limit_ns)
+            : mbar_wait(&bars[kBarPVLast], 0, s_abort, P.wait_limit_ns);
+        ok = __all_sync(0xffffffffu, w) && ok;
+        tc_fence_after();
         const float a = resc ? exp2f(m_run - m_new) : 1.f;
 #pragma unroll
         for (int ch = 0; ch < HD / 32; ++ch) {
@@ -610,40 +607,34 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       const float mref = (m_new == -INFINITY) ? 0.f : m_new;
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
       float2 ps0 = make_float2(0.f, 0.f), ps1 = make_float2(0.f, 0.f);
-      // probabilities per 64-key half (published separately so that the PV MMAs of the
-      // first half overlap the exponentials of the second), in chunks of 32 keys packed to
-      // bf16 pairs and stored to tensor memory (16 columns) at once.  A half with no valid
-      // key for this row (warp-uniform) is written as zeros without exponentials.
+      // probabilities in chunks of 32 keys packed to bf16 pairs and stored to tensor memory
+      // (16 columns) at once; with no valid key for this row (warp-uniform) the chunk is
+      // written as zeros without exponentials
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const bool any = (hf == 0 ? v0 : v1) > 0;
+      for (int ch = 0; ch < 2; ++ch) {
+        float pk[16];
+        if (v > 0) {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int ch = hf * 2 + cc;
-          float pk[16];
-          if (any) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int i0 = ch * 32 + 2 * e;
-              const float2 x = ffma2(make_float2(sv[i0], sv[i0 + 1]), c2, nm2);
-              float2 p;
-              p.x = ex2_approx(x.x);
-              p.y = ex2_approx(x.y);
-              if (e & 1) ps1 = fadd2(ps1, p); else ps0 = fadd2(ps0, p);
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
-              pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&b2));
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = 0.f;
+          for (int e = 0; e < 16; ++e) {
+            const int i0 = ch * 32 + 2 * e;
+            const float2 x = ffma2(make_float2(sv[i0], sv[i0 + 1]), c2, nm2);
+            float2 p;
+            p.x = ex2_approx(x.x);
+            p.y = ex2_approx(x.y);
+            if (e & 1) ps1 = fadd2(ps1, p); else ps0 = fadd2(ps0, p);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
+            pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&b2));
           }
-          tmem_st16(t_row + s_col + ch * 16, pk);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0.f;
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarPFull + 2 * wg + hf]);
+        tmem_st16(t_row + s_col + ch * 16, pk);
       }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarPFull + 2 * sb + wg]);
       if (threadIdx.x == 128) LF_TR(10, l);
       l_run += (ps0.x + ps0.y) + (ps1.x + ps1.y);
       m_run = m_new;
