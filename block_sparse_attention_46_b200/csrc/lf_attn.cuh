@@ -282,6 +282,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   float* s_red = reinterpret_cast<float*>(smem + L::kRed);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* s_stop = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);   // producers' ends
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -415,27 +416,44 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
 
   if (warp < 4) {
   regs_dec<kLowRegs>();
-  // -------------------------------------------------------------- producer
-  if (warp == 0 && lane == 0) {
+  // -------------------------------------------------------------- producers
+  // Two threads issue the loads: warp 0 the K tiles, warp 2 the V tiles, each in ring order
+  // within its own positions (a single thread issuing both cannot keep the ring filled
+  // ahead of the MMAs on gathered key blocks).
+  if (warp == 0 || warp == 2) {
     uint64_t* full = &bars[kBarRing];
     uint64_t* empty = &bars[kBarRing + L::kSlots];
     const int n_pos = 2 * n_iter + 1;               // V of the last tile sits at 2n
-    int q = pre;                                    // positions loaded in the set-up
-    for (; q < n_pos; ++q) {
-      bool isK;
-      const int l = ring_tile(q, isK);
-      const int slot = q % L::kSlots;
-      const int rnd = q / L::kSlots;
-      if (isK && l >= n_iter) continue;            // no slot used, nothing to load
-      if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort, P.wait_limit_ns)) break;
-      load_pos(q, isK, l);
+    const bool kside = warp == 0;
+    if (lane == 0) {
+      int q = kside ? pre : 2;                      // K positions below pre went in the set-up
+      for (; q < n_pos; ++q) {
+        bool isK;
+        const int l = ring_tile(q, isK);
+        if (isK != kside || (isK && l >= n_iter)) continue;   // the other side's, or no load
+        const int slot = q % L::kSlots;
+        const int rnd = q / L::kSlots;
+        if (rnd > 0 && !mbar_wait(&empty[slot], (rnd & 1) ^ 1, s_abort, P.wait_limit_ns)) break;
+        load_pos(q, isK, l);
+      }
+      s_stop[kside ? 0 : 1] = q;                    // positions of this side below q issued
     }
-    // drain: every load issued must land before the CTA may exit (the last kSlots
-    // positions hold the only loads that nobody may have waited for)
-    for (int x = max(0, q - L::kSlots); x < q; ++x) {
-      bool isK;
-      const int lx = ring_tile(x, isK);
-      if (!(isK && lx >= n_iter)) mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1, P.wait_limit_ns);
+    __syncwarp();
+    named_bar_sync(2, 64);
+    // drain: every load issued must land before the CTA may exit.  A load whose slot was
+    // issued again (position + kSlots) is known to have landed; the others are waited for.
+    if (warp == 0 && lane == 0) {
+      const int qk = s_stop[0], qv = s_stop[1];
+      auto issued = [&](int x) {
+        if (x >= n_pos) return false;
+        bool isK;
+        const int lx = ring_tile(x, isK);
+        if (isK && lx >= n_iter) return false;
+        return x < (isK ? qk : qv);
+      };
+      for (int x = max(0, min(qk, qv) - 2 * L::kSlots); x < max(qk, qv); ++x)
+        if (issued(x) && !issued(x + L::kSlots))
+          mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1, P.wait_limit_ns);
     }
   }
   // -------------------------------------------------------------- MMA issuer
