@@ -15,12 +15,12 @@
 //   * the key plan of a tile (sink blocks, then the sorted union of its query blocks'
 //     selected blocks, each with a bit per query block that selected it) is built by
 //     plan_kernel; a key column a row's query block did not select is masked to -inf;
-//   * warp 0 streams Q, then K and V tiles, with TMA (128-byte swizzle, zero fill out of
-//     bounds) into one ring of 160 KB (five 32 KB stages at d = 128) in the order the MMAs
-//     consume them; warp 1 issues tcgen05.mma: S = Q K^T into one of two tensor-memory
-//     buffers (S of tile l+1 is computed while the softmax works on tile l), and per
-//     softmax warpgroup O_w += P_w V_w over that warpgroup's 64 keys of the tile; warp 3
-//     stages the tile's key plan into shared memory;
+//   * Q, then K and V tiles, stream with TMA (128-byte swizzle, zero fill out of bounds)
+//     into one ring of 160 KB (five 32 KB stages at d = 128) in the order the MMAs consume
+//     them, the K tiles issued by warp 0 and the V tiles by warp 2; warp 1 issues the
+//     tcgen05.mma S = Q K^T into one of two tensor-memory buffers (S of tile l+1 is computed
+//     while the softmax works on tile l) and warp 3, once it has staged the tile's key plan
+//     into shared memory, the PVs: O_w += P_w V_w over softmax warpgroup w's 64 keys;
 //   * warps 4-11 are two softmax warpgroups; warpgroup w takes keys [64w, 64w + 64) of
 //     every key tile and keeps its own fp32 online softmax state and O_w over them, one
 //     query row per thread (the row's tensor-memory lane): S from tensor memory, P as bf16
@@ -206,8 +206,9 @@ struct AttnParams {
 
 // barrier indices: ring full/empty barriers follow these
 // P barriers: kBarPFull + 2 * buffer + warpgroup (keys 0-63, 64-127 of the tile)
-// kBarPVLast: completion of the PVs of the last tile but one (committed once)
-enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 7, kBarPVLast = 8, kBarRing = 9 };
+// PV barriers: kBarPVDone + buffer, completion of both PVs of a tile
+// kBarDone: completion of everything the two MMA threads issued (one arrival each)
+enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 7, kBarPVDone = 8, kBarRing = 10 };
 
 template <int HD>
 struct AttnLayout {
@@ -388,8 +389,9 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       mbar_init(&bars[kBarPFull + 2 * s + 1], 4);
     }
     for (int q = 0; q < 2 * L::kSlots; ++q) mbar_init(&bars[kBarRing + q], 1);
-    mbar_init(&bars[kBarDone], 1);
-    mbar_init(&bars[kBarPVLast], 1);
+    mbar_init(&bars[kBarDone], 2);
+    mbar_init(&bars[kBarPVDone], 1);
+    mbar_init(&bars[kBarPVDone + 1], 1);
     *s_abort = 0;
     fence_mbar_init();
     // Q and the first key tiles when they are dense (no key plan needed) go out now, so
@@ -456,75 +458,78 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
           mbar_wait_drain(&full[x % L::kSlots], (x / L::kSlots) & 1, P.wait_limit_ns);
     }
   }
-  // -------------------------------------------------------------- MMA issuer
-  // Order: S0, S1, then for each l: PV_l of warpgroup 0 and of warpgroup 1 (O_w += P_w V_w,
-  // the warpgroup's 64 keys of tile l), S_{l+2} into the S buffer P_l was read from.
-  // tcgen05.mma runs in issue order, so S_{l+2} overwrites P_l only after both PVs have
-  // consumed it, and the completion of S_{l+1} implies that of PV_{l-1}.
-  else if (warp == 1 && lane == 0) {
+  // -------------------------------------------------------------- MMA issuers
+  // Two threads issue tcgen05.mma: warp 1 S_l = Q K_l^T into S buffer l & 1, warp 3 the PVs
+  // of tile l (O_w += P_w V_w, warpgroup w's 64 keys) as soon as each warpgroup's P is
+  // written.  S_{l+2} overwrites P_l, so it is issued only after both PVs of tile l have
+  // completed (PV barrier of the buffer); the PV thread is never held up behind S MMAs.
+  else if ((warp == 1 || warp == 3) && lane == 0) {
     constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, 0, 1);
     const uint32_t q_base = smem_u32(smem + L::kQ);
     const uint32_t ring_base = smem_u32(smem + L::kRing);
     uint64_t* full = &bars[kBarRing];
     uint64_t* empty = &bars[kBarRing + L::kSlots];
-    auto issue_s = [&](int l) -> bool {
-      const int s = l & 1;
-      const int q = ring_pos_k(l), slot = q % L::kSlots;
-      LF_TR(2, l);
-      if (!mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort, P.wait_limit_ns)) return false;
-      LF_TR(3, l);
-      tc_fence_after();
-      const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
-      const uint32_t k_addr = ring_base + slot * L::kStageBytes;
-      if constexpr (F8) {
-#pragma unroll
-        for (int ks = 0; ks < HD / 32; ++ks)          // 32 e4m3 elements = 32 bytes per MMA
-          mma_e4m3_ss(d_tmem, smem_desc_sw128(q_base + ks * 32, 16, 1024),
-                      smem_desc_sw128(k_addr + ks * 32, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
-      } else {
-#pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
-          mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
-                      smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
-        }
-      }
-      mma_commit(&bars[kBarSFull + s]);
-      mma_commit(&empty[slot]);
-      return true;
-    };
-    bool ok = mbar_wait(&bars[kBarQ], 0, s_abort, P.wait_limit_ns);
-    if (ok && n_iter > 0) ok = issue_s(0);
-    if (ok && n_iter > 1) ok = issue_s(1);
-    for (int l = 0; ok && l < n_iter; ++l) {
-      const int s = l & 1;
-      const int qv = ring_pos_v(l), vslot = qv % L::kSlots;
-      ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort, P.wait_limit_ns);
-      LF_TR(4, l);
-      const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
-      // each warpgroup's P (its 64 keys) goes into its own O as soon as it is written
-      for (int wg = 0; ok && wg < 2; ++wg) {
-        ok = mbar_wait(&bars[kBarPFull + 2 * s + wg], (l >> 1) & 1, s_abort, P.wait_limit_ns);
+    bool ok = true;
+    if (warp == 1) {
+      ok = mbar_wait(&bars[kBarQ], 0, s_abort, P.wait_limit_ns);
+      for (int l = 0; ok && l < n_iter; ++l) {
+        const int s = l & 1;
+        // P_{l-2} (over this buffer) consumed: the PVs of tile l-2 completed
+        if (l >= 2) ok = mbar_wait(&bars[kBarPVDone + s], ((l >> 1) & 1) ^ 1, s_abort, P.wait_limit_ns);
+        const int q = ring_pos_k(l), slot = q % L::kSlots;
+        LF_TR(2, l);
+        if (ok) ok = mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort, P.wait_limit_ns);
         if (!ok) break;
-        if (wg == 0) LF_TR(5, l);
+        LF_TR(3, l);
         tc_fence_after();
-        const uint32_t o_tmem = tmem + (wg ? L::kColO1 : L::kColO0);
+        const uint32_t d_tmem = tmem + (s ? L::kColS1 : L::kColS0);
+        const uint32_t k_addr = ring_base + slot * L::kStageBytes;
+        if constexpr (F8) {
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {        // 16 keys per MMA, 8 P columns each
-          const int ks = wg * 4 + k4;           // 16-key step within the V tile
-          mma_bf16_ts(o_tmem, p_tmem + wg * 64 + k4 * 8,
-                      smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
-                                      L::kRegion, 1024),
-                      idesc_pv, (l > 0 || k4 > 0) ? 1u : 0u);
+          for (int ks = 0; ks < HD / 32; ++ks)          // 32 e4m3 elements = 32 bytes per MMA
+            mma_e4m3_ss(d_tmem, smem_desc_sw128(q_base + ks * 32, 16, 1024),
+                        smem_desc_sw128(k_addr + ks * 32, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < HD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * L::kRegion + (ks & 3) * 32;
+            mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
+                        smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+          }
         }
+        mma_commit(&bars[kBarSFull + s]);
+        mma_commit(&empty[slot]);
       }
-      if (!ok) break;
-      mma_commit(&empty[vslot]);
-      if (l + 2 < n_iter) ok = issue_s(l + 2);
-      else if (l + 2 == n_iter) mma_commit(&bars[kBarPVLast]);   // no S_{l+2} to imply it
+    } else {
+      for (int l = 0; ok && l < n_iter; ++l) {
+        const int s = l & 1;
+        const int qv = ring_pos_v(l), vslot = qv % L::kSlots;
+        ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort, P.wait_limit_ns);
+        LF_TR(4, l);
+        const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
+        for (int wg = 0; ok && wg < 2; ++wg) {
+          ok = mbar_wait(&bars[kBarPFull + 2 * s + wg], (l >> 1) & 1, s_abort, P.wait_limit_ns);
+          if (!ok) break;
+          if (wg == 0) LF_TR(5, l);
+          tc_fence_after();
+          const uint32_t o_tmem = tmem + (wg ? L::kColO1 : L::kColO0);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {        // 16 keys per MMA, 8 P columns each
+            const int ks = wg * 4 + k4;           // 16-key step within the V tile
+            mma_bf16_ts(o_tmem, p_tmem + wg * 64 + k4 * 8,
+                        smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
+                                        L::kRegion, 1024),
+                        idesc_pv, (l > 0 || k4 > 0) ? 1u : 0u);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&empty[vslot]);
+        mma_commit(&bars[kBarPVDone + s]);
+      }
     }
-    // completion of everything issued: epilogue may read O, tensor memory may be freed
+    // completion of everything this thread issued: epilogue may read O, tensor memory may
+    // be freed once both threads' arrivals are in
     mma_commit(&bars[kBarDone]);
   }
   } else {
@@ -599,13 +604,10 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       float m_new = m_run;
       bool resc = false;
       if (m_tile > m_run + 8.0f) { m_new = m_tile; resc = true; }
-      // lazy rescale of this group's O.  Its last PV (PV_{l-1}) was issued after S_l, so it
-      // is waited for: it completed before S_{l+1} did, or, when l is the last tile, before
-      // the commit that follows it.
+      // lazy rescale of this group's O, once its last PV (PV_{l-1}) has completed
       if (l > 0 && __any_sync(0xffffffffu, resc)) {
-        const bool w = l + 1 < n_iter
-            ? mbar_wait(&bars[kBarSFull + (sb ^ 1)], ((l + 1) >> 1) & 1, s_abort, P.wait_limit_ns)
-            : mbar_wait(&bars[kBarPVLast], 0, s_abort, P.wait_limit_ns);
+        const bool w = mbar_wait(&bars[kBarPVDone + (sb ^ 1)], ((l - 1) >> 1) & 1, s_abort,
+                                 P.wait_limit_ns);
         ok = __all_sync(0xffffffffu, w) && ok;
         tc_fence_after();
         const float a = resc ? exp2f(m_run - m_new) : 1.f;
