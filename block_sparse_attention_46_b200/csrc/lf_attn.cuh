@@ -475,11 +475,12 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       ok = mbar_wait(&bars[kBarQ], 0, s_abort, P.wait_limit_ns);
       for (int l = 0; ok && l < n_iter; ++l) {
         const int s = l & 1;
-        // P_{l-2} (over this buffer) consumed: the PVs of tile l-2 completed
-        if (l >= 2) ok = mbar_wait(&bars[kBarPVDone + s], ((l >> 1) & 1) ^ 1, s_abort, P.wait_limit_ns);
         const int q = ring_pos_k(l), slot = q % L::kSlots;
         LF_TR(2, l);
-        if (ok) ok = mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort, P.wait_limit_ns);
+        // K_l (which lands early), then P_{l-2} (over this buffer) consumed: the PVs of tile
+        // l-2 completed, the wait the issue depends on
+        ok = mbar_wait(&full[slot], (q / L::kSlots) & 1, s_abort, P.wait_limit_ns);
+        if (ok && l >= 2) ok = mbar_wait(&bars[kBarPVDone + s], ((l >> 1) & 1) ^ 1, s_abort, P.wait_limit_ns);
         if (!ok) break;
         LF_TR(3, l);
         tc_fence_after();
@@ -524,8 +525,8 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
           }
         }
         if (!ok) break;
-        mma_commit(&empty[vslot]);
         mma_commit(&bars[kBarPVDone + s]);
+        mma_commit(&empty[vslot]);
       }
     }
     // completion of everything this thread issued: epilogue may read O, tensor memory may
