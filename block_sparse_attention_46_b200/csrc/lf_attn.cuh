@@ -205,10 +205,15 @@ struct AttnParams {
 };
 
 // barrier indices: ring full/empty barriers follow these
-// P barriers: kBarPFull + 2 * buffer + warpgroup (keys 0-63, 64-127 of the tile)
 // PV barriers: kBarPVDone + buffer, completion of both PVs of a tile
 // kBarDone: completion of everything the two MMA threads issued (one arrival each)
-enum BarId { kBarQ = 0, kBarSFull = 1, kBarPFull = 3, kBarDone = 7, kBarPVDone = 8, kBarRing = 10 };
+enum BarId { kBarQ = 0, kBarSFull = 1, kBarDone = 3, kBarPVDone = 4, kBarRing = 6 };
+// named barriers (0 is __syncthreads): the epilogue's exchange, the producers' drain, and
+// per softmax warpgroup w the hand-off of each tile's P to the PV thread's warp.  Both
+// sides wait (bar.sync) once per tile, so no warp can arrive for a later tile before a
+// tile's hand-off is complete, also when an aborted wait has desynchronised the loops.
+constexpr int kNbEpilogue = 1, kNbProducers = 2, kNbP = 3;   // kNbP + w
+constexpr int kNbPThreads = 160;                              // 4 softmax warps + PV warp
 
 template <int HD>
 struct AttnLayout {
@@ -385,8 +390,6 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     mbar_init(&bars[kBarQ], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kBarSFull + s], 1);
-      mbar_init(&bars[kBarPFull + 2 * s], 4);
-      mbar_init(&bars[kBarPFull + 2 * s + 1], 4);
     }
     for (int q = 0; q < 2 * L::kSlots; ++q) mbar_init(&bars[kBarRing + q], 1);
     mbar_init(&bars[kBarDone], 2);
@@ -441,7 +444,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       s_stop[kside ? 0 : 1] = q;                    // positions of this side below q issued
     }
     __syncwarp();
-    named_bar_sync(2, 64);
+    named_bar_sync(kNbProducers, 64);
     // drain: every load issued must land before the CTA may exit.  A load whose slot was
     // issued again (position + kSlots) is known to have landed; the others are waited for.
     if (warp == 0 && lane == 0) {
@@ -463,7 +466,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
   // of tile l (O_w += P_w V_w, warpgroup w's 64 keys) as soon as each warpgroup's P is
   // written.  S_{l+2} overwrites P_l, so it is issued only after both PVs of tile l have
   // completed (PV barrier of the buffer); the PV thread is never held up behind S MMAs.
-  else if ((warp == 1 || warp == 3) && lane == 0) {
+  else if (warp == 1 || warp == 3) {
     constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, 0, 1);
     const uint32_t q_base = smem_u32(smem + L::kQ);
@@ -471,7 +474,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     uint64_t* full = &bars[kBarRing];
     uint64_t* empty = &bars[kBarRing + L::kSlots];
     bool ok = true;
-    if (warp == 1) {
+    if (warp == 1 && lane == 0) {
       ok = mbar_wait(&bars[kBarQ], 0, s_abort, P.wait_limit_ns);
       for (int l = 0; ok && l < n_iter; ++l) {
         const int s = l & 1;
@@ -502,36 +505,41 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
         mma_commit(&bars[kBarSFull + s]);
         mma_commit(&empty[slot]);
       }
-    } else {
-      for (int l = 0; ok && l < n_iter; ++l) {
+    } else if (warp == 3) {
+      // every iteration meets both warpgroups at their barriers, also after a failed wait,
+      // so that the syncs on each named barrier stay paired
+      for (int l = 0; l < n_iter; ++l) {
         const int s = l & 1;
         const int qv = ring_pos_v(l), vslot = qv % L::kSlots;
-        ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort, P.wait_limit_ns);
-        LF_TR(4, l);
+        if (lane == 0 && ok) ok = mbar_wait(&full[vslot], (qv / L::kSlots) & 1, s_abort, P.wait_limit_ns);
+        if (lane == 0) LF_TR(4, l);
         const uint32_t p_tmem = tmem + (s ? L::kColS1 : L::kColS0);
-        for (int wg = 0; ok && wg < 2; ++wg) {
-          ok = mbar_wait(&bars[kBarPFull + 2 * s + wg], (l >> 1) & 1, s_abort, P.wait_limit_ns);
-          if (!ok) break;
-          if (wg == 0) LF_TR(5, l);
-          tc_fence_after();
-          const uint32_t o_tmem = tmem + (wg ? L::kColO1 : L::kColO0);
+        for (int wg = 0; wg < 2; ++wg) {
+          __syncwarp();
+          named_bar_sync(kNbP + wg, kNbPThreads);            // P_l of warpgroup wg written
+          if (lane == 0 && ok) {
+            if (wg == 0) LF_TR(5, l);
+            tc_fence_after();
+            const uint32_t o_tmem = tmem + (wg ? L::kColO1 : L::kColO0);
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {        // 16 keys per MMA, 8 P columns each
-            const int ks = wg * 4 + k4;           // 16-key step within the V tile
-            mma_bf16_ts(o_tmem, p_tmem + wg * 64 + k4 * 8,
-                        smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
-                                        L::kRegion, 1024),
-                        idesc_pv, (l > 0 || k4 > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < 4; ++k4) {        // 16 keys per MMA, 8 P columns each
+              const int ks = wg * 4 + k4;           // 16-key step within the V tile
+              mma_bf16_ts(o_tmem, p_tmem + wg * 64 + k4 * 8,
+                          smem_desc_sw128(ring_base + vslot * L::kStageBytes + ks * 16 * 128,
+                                          L::kRegion, 1024),
+                          idesc_pv, (l > 0 || k4 > 0) ? 1u : 0u);
+            }
           }
         }
-        if (!ok) break;
-        mma_commit(&bars[kBarPVDone + s]);
-        mma_commit(&empty[vslot]);
+        if (lane == 0 && ok) {
+          mma_commit(&bars[kBarPVDone + s]);
+          mma_commit(&empty[vslot]);
+        }
       }
     }
     // completion of everything this thread issued: epilogue may read O, tensor memory may
     // be freed once both threads' arrivals are in
-    mma_commit(&bars[kBarDone]);
+    if (lane == 0) mma_commit(&bars[kBarDone]);
   }
   } else {
   regs_inc<kHighRegs>();
@@ -654,8 +662,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
       }
       tmem_st_wait();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarPFull + 2 * sb + wg]);
+      named_bar_sync(kNbP + wg, kNbPThreads);              // hand P_l to the PV thread
       if (threadIdx.x == 128) LF_TR(10, l);
       l_run += (ps0.x + ps0.y) + (ps1.x + ps1.y);
       m_run = m_new;
@@ -665,7 +672,7 @@ attn_kernel(const __grid_constant__ AttnParams P, const Dims D) {
     // merge the two groups' partial softmax states: O = sum_w 2^(m_w - m) O_w / l
     s_red[wg * 128 + r] = m_run;
     s_red[256 + wg * 128 + r] = l_run;
-    named_bar_sync(1, kSoftmaxWarps * 32);
+    named_bar_sync(kNbEpilogue, kSoftmaxWarps * 32);
     const float m_o = s_red[(wg ^ 1) * 128 + r], l_o = s_red[256 + (wg ^ 1) * 128 + r];
     const float m_all = fmaxf(m_run, m_o);
     const float w_me = m_run == -INFINITY ? 0.f : exp2f(m_run - m_all);
