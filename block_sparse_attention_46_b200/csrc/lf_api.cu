@@ -699,9 +699,9 @@ int lf_quantize_e4m3(const void* x, int64_t rows, int32_t H, int32_t d, const fl
       (head_scale == nullptr && (row_scale == nullptr || !aligned(row_scale, 4))) ||
       (head_scale != nullptr && !aligned(head_scale, 4)))
     return LF_ERR_INVALID_ARG;
-  const long long units = rows * H;
-  const int warps = 8;
-  lf::quantize_e4m3_kernel<<<(unsigned)((units + warps - 1) / warps), warps * 32, 0, stream>>>(
+  const long long threads = rows * H * (d / 8);   // d / 8 threads per (row, head)
+  const int block = 256;
+  lf::quantize_e4m3_kernel<<<(unsigned)((threads + block - 1) / block), block, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(x), rows, H, d, head_scale, x8, row_scale);
   return cuda_status(cudaGetLastError());
 }

@@ -30,45 +30,50 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
 
 // x [rows, H, d] bf16 -> x8 [rows, H, d] e4m3 codes.  head_scale != null: one given scale per
 // head; else a scale per (row, head) computed here and written to row_scale [rows, H].
-// One warp per (row, head); d / 32 channels per lane (d in {64, 128}).
+// d / 8 threads per (row, head), eight channels each (one 16-byte load, one 8-byte store);
+// a (row, head)'s threads are consecutive lanes of one warp, which reduce its max |x|.
 __global__ void quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ x, long long rows, int H,
                                      int d, const float* __restrict__ head_scale,
                                      uint8_t* __restrict__ x8, float* __restrict__ row_scale) {
-  const long long unit = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (unit >= rows * H) return;
+  const int tpu = d / 8;                          // 16 or 8 threads per (row, head)
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long unit = gt / tpu;
+  const int sub = (int)(gt % tpu);
+  const bool valid = unit < rows * H;             // the others only join the shuffles
   const int h = (int)(unit % H);
-  const int per = d / 32;                         // 2 or 4 channels per lane
-  const __nv_bfloat16* src = x + unit * d + lane * per;
-  float v[4];
-  if (per == 4) {                                  // one 8-byte load (rows are 16-byte aligned)
-    const uint2 u = *reinterpret_cast<const uint2*>(src);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  float v[8];
+  if (valid) {
+    const uint4 u = *reinterpret_cast<const uint4*>(x + unit * d + sub * 8);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
   } else {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src));
-    v[0] = a.x; v[1] = a.y;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
   }
   float scale;
   if (head_scale != nullptr) {
-    scale = head_scale[h];
+    scale = valid ? head_scale[h] : 1.f;
   } else {
     float a = 0.f;
-    for (int i = 0; i < per; ++i) a = fmaxf(a, fabsf(v[i]));
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    for (int o = tpu / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     scale = ldexpf(1.0f, pow2_exponent(a));
-    if (lane == 0) row_scale[unit] = scale;
+    if (valid && sub == 0) row_scale[unit] = scale;
   }
+  if (!valid) return;
   const float inv = 1.0f / scale;                 // exact: a power of two
-  uint8_t* dst = x8 + unit * d + lane * per;
-  const uint16_t c01 = cvt_e4m3x2(v[0] * inv, v[1] * inv);
-  if (per == 4) {                                  // the lane's four codes in one store
-    const uint16_t c23 = cvt_e4m3x2(v[2] * inv, v[3] * inv);
-    *reinterpret_cast<uint32_t*>(dst) = (uint32_t)c01 | ((uint32_t)c23 << 16);
-  } else {
-    *reinterpret_cast<uint16_t*>(dst) = c01;
-  }
+  uint32_t c[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    c[i] = (uint32_t)cvt_e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv) |
+           ((uint32_t)cvt_e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv) << 16);
+  *reinterpret_cast<uint2*>(x8 + unit * d + sub * 8) = make_uint2(c[0], c[1]);
 }
 
 // Per-head max |x| over rows x d, folded into amax_bits[h] (non-negative floats order like
