@@ -7,8 +7,9 @@ model keeps the kernel's barrier counts and the parity each wait uses:
 
 * mbarriers complete a phase when their arrivals (and, for a TMA fill, its bytes) are in;
   ``try_wait.parity(p)`` succeeds when the barrier's completed-phase count has the other
-  parity.  Every wait also records which phase it meant, so a waiter that is two phases
-  behind (the case where a parity wait returns at once by mistake) is reported.
+  parity.  Every wait also records which phase it meant, so a wait that passes for the
+  wrong phase (its waiter two phases behind, or two phases ahead of the barrier, where the
+  parity looks the same) is reported.
 * a tcgen05.commit arrives when every MMA its thread issued before it has completed; MMAs
   of one thread run in issue order, MMAs of different threads in any order.
 * named barriers (bar.sync) complete a generation when all participants have arrived.
@@ -91,11 +92,15 @@ class Sim:
             b[1] = b[0]
 
     def test(self, name, phase):
-        """try_wait.parity for the phase index the caller means."""
+        """try_wait.parity for the phase index the caller means.  The parity answers right
+        only while the barrier has completed phase - 1 or phase (or phase + 1 phases in
+        all); a wait outside that window is reported."""
         done = self.bars[name][2]
         ok = (done & 1) != (phase & 1)
         if ok and done > phase + 1:
             self.issues.append(f"{name}: waiter of phase {phase} is {done - phase} phases behind")
+        if ok and done < phase + 1:
+            self.issues.append(f"{name}: wait for phase {phase} passed with {done} phases done")
         return ok
 
     def later(self, dt, fn):
